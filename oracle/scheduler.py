@@ -1,0 +1,77 @@
+"""CPU restatement of the split-KV work partition (TEST INFRASTRUCTURE ONLY).
+
+The pages ask for a decode kernel optimised for serving variable-length
+sequences ("OpenSourceWeek Day 1: FlashMLA", opening paragraph; "DeepSeek
+merilis open source FlashMLA", release bullets) but print no partition rule.  The rule below is the
+one the library documents in its header, restated independently in plain
+Python loops so that the GPU's metadata can be compared with it bit for bit:
+
+  n_i     = ceil(L_i / 64) pages of sequence i
+  items_i = max(n_i, 1)        (an empty sequence still owns one item: its
+                                 output, zeros and lse = -inf, must be written)
+  every sequence costs PIECE_COST + items_i units; laid end to end, sequence i
+  starts at unit start_i and its item j sits at unit start_i + PIECE_COST + j.
+  cap     = ceil(total / W);  the item at unit u belongs to worker u // cap.
+
+A worker therefore owns one contiguous run of items, which may begin or end
+inside a sequence.  A sequence spread over k workers yields k pieces ("splits")
+that are merged afterwards by log-sum-exp.
+
+Per worker the metadata row holds 8 int32:
+  [begin_seq, begin_item, end_seq, end_item (exclusive), begin_split, num_pieces, 0, 0]
+with num_pieces = 0 (and the rest 0) for a worker that owns nothing.
+num_splits[i + 1] - num_splits[i] is the number of pieces of sequence i.
+"""
+from __future__ import annotations
+
+PAGE = 64
+PIECE_COST = 2
+MD_STRIDE = 8
+
+
+def split_plan(seqlens, num_workers: int):
+    """Returns (tile_md as a list of num_workers rows of 8 ints, num_splits list of b+1)."""
+    lens = [int(v) for v in seqlens]
+    W = int(num_workers)
+    assert W >= 1
+    items = []
+    for L in lens:
+        n = (L + PAGE - 1) // PAGE if L > 0 else 0
+        items.append(max(n, 1))
+    starts = []
+    total = 0
+    for it in items:
+        starts.append(total)
+        total += PIECE_COST + it
+    cap = max(1, -(-total // W))
+
+    # which worker owns each item, written out item by item
+    owner = {}
+    for i, it in enumerate(items):
+        for j in range(it):
+            owner[(i, j)] = (starts[i] + PIECE_COST + j) // cap
+
+    md = [[0] * MD_STRIDE for _ in range(W)]
+    pieces_of_seq = [0] * len(lens)
+    first_worker_of_seq = [None] * len(lens)
+    for i, it in enumerate(items):
+        ws = sorted({owner[(i, j)] for j in range(it)})
+        pieces_of_seq[i] = len(ws)
+        first_worker_of_seq[i] = ws[0]
+    for w in range(W):
+        mine = [(i, j) for i, it in enumerate(items) for j in range(it) if owner[(i, j)] == w]
+        if not mine:
+            continue
+        (bs, bi), (es, ei) = mine[0], mine[-1]
+        n_pieces = len({i for i, _ in mine})
+        md[w] = [bs, bi, es, ei + 1, w - first_worker_of_seq[bs], n_pieces, 0, 0]
+    num_splits = [0]
+    for k in pieces_of_seq:
+        num_splits.append(num_splits[-1] + k)
+    return md, num_splits
+
+
+def num_workers_for(num_sms: int, s_q: int, h_q: int, rows_per_cta: int = 64) -> int:
+    """Workers the decode grid uses: one CTA per SM, shared among the row blocks."""
+    row_blocks = -(-(s_q * h_q) // rows_per_cta)
+    return max(1, num_sms // row_blocks)

@@ -1,0 +1,99 @@
+"""Pins for the CPU restatement of the split-KV partition rule (no GPU).
+
+The rule is the library's own design (the pages print none), so these checks
+fix what any correct partition must satisfy, and brute force over small cases.
+"""
+import itertools
+
+import pytest
+
+from oracle.scheduler import PAGE, PIECE_COST, split_plan
+
+
+def items_of(L):
+    return max((L + PAGE - 1) // PAGE, 1)
+
+
+def check_plan(lens, W):
+    md, ns = split_plan(lens, W)
+    b = len(lens)
+    assert len(md) == W and len(ns) == b + 1 and ns[0] == 0
+    # every item of every sequence is covered exactly once, workers in order
+    seen = {}
+    pieces = {i: [] for i in range(b)}
+    order = []
+    for w, row in enumerate(md):
+        bs, bi, es, ei, bsplit, npieces = row[:6]
+        assert row[6] == 0 and row[7] == 0
+        if npieces == 0:
+            assert row == [0] * 8
+            continue
+        assert npieces == es - bs + 1 and bs <= es
+        for i in range(bs, es + 1):
+            lo = bi if i == bs else 0
+            hi = ei if i == es else items_of(lens[i])
+            assert 0 <= lo < hi <= items_of(lens[i])
+            for j in range(lo, hi):
+                assert (i, j) not in seen
+                seen[(i, j)] = w
+                order.append((i, j))
+            pieces[i].append((w, lo, hi))
+    assert len(seen) == sum(items_of(L) for L in lens)
+    assert order == sorted(order)  # contiguous, lexicographic runs
+    for i in range(b):
+        k = ns[i + 1] - ns[i]
+        assert k == len(pieces[i]) and k >= 1
+        # split indices: the worker that starts a sequence has split 0, the next 1, ...
+        for s, (w, lo, hi) in enumerate(pieces[i]):
+            expect = md[w][4] if md[w][0] == i else 0
+            assert s == expect
+    # balance: no worker owns more than cap items
+    total = sum(PIECE_COST + items_of(L) for L in lens)
+    cap = -(-total // W)
+    for w in range(W):
+        assert sum(1 for v in seen.values() if v == w) <= cap
+    # pieces beyond one per sequence come only from worker boundaries
+    assert ns[-1] <= b + W - 1
+    return md, ns
+
+
+def test_single_worker_takes_everything():
+    md, ns = check_plan([37, 130, 0], 1)
+    assert md[0][:6] == [0, 0, 2, 1, 0, 3]
+    assert ns == [0, 1, 2, 3]
+
+
+def test_one_sequence_per_worker_when_costs_align():
+    # 4 sequences of 6 pages each, cost 8 units each, 4 workers: one each, no splits
+    md, ns = check_plan([6 * 64] * 4, 4)
+    assert ns == [0, 1, 2, 3, 4]
+    assert [r[:6] for r in md] == [[i, 0, i, 6, 0, 1] for i in range(4)]
+
+
+def test_long_sequence_is_split_across_workers():
+    md, ns = check_plan([32768] * 15 + [1], 74)
+    assert ns[-1] > 16                  # the long sequences are cut
+    assert ns[16] - ns[15] == 1         # the one-token sequence is whole
+
+
+def test_more_workers_than_items():
+    md, ns = check_plan([37, 130], 148)
+    assert sum(1 for r in md if r[5] > 0) == 4   # one worker per page
+    assert ns == [0, 1, 4]
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 5, 7])
+def test_brute_force_small(W):
+    lengths = [0, 1, 63, 64, 65, 128, 129, 300]
+    for b in (1, 2, 3):
+        for lens in itertools.product(lengths, repeat=b):
+            check_plan(list(lens), W)
+
+
+def test_realistic_shapes():
+    import torch
+    g = torch.Generator().manual_seed(0)
+    for W in (37, 74, 148):
+        lens = torch.randint(1, 8193, (128,), generator=g).tolist()
+        check_plan(lens, W)
+        check_plan([4096] * 64, W)
