@@ -1,0 +1,152 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) MLA paged latent-cache decoder.
+ *
+ * The operation ("OpenSourceWeek Day 1: FlashMLA", opening paragraph and "Key
+ * Highlights"; "FlashMLA: Revolutionizing Efficient Decoding in Large Language
+ * Models...", sections 4.1.1 and 4.3.2): multi-head latent attention decoding.
+ * Every query head attends over one cached latent row per token, shared by all
+ * heads ("How MLA Optimizes Memory Usage": only c_t is cached and both K and V
+ * derive from it).  Rows are bf16 and live in 64-token pages reached through a
+ * per-sequence block table.  For sequence i, query position j and head h:
+ *
+ *     s_t   = softmax_scale * <q[i][j][h][0:576], K_t[0:576]>   for visible t
+ *     out   = sum_t softmax(s)_t * K_t[0:512]       (the value is the first 512 dims)
+ *     lse   = ln sum_t exp(s_t)
+ *
+ * with K_t = kcache[block_table[i][t / 64]][t % 64].  Visible tokens are
+ * t < cache_seqlens[i]; with `causal`, query j (of s_q) sees t <= L - s_q + j
+ * (the s_q queries are the last s_q positions).  An empty visible set yields
+ * out = 0 and lse = -inf.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are caller-owned device memory; the library allocates no
+ *     device memory and keeps no state beyond a per-device cache of SM counts
+ *     and kernel attributes.  Tensors are contiguous and row-major with the
+ *     shapes stated.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronises.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failing check returns MLA_ERR_INVALID_ARG or MLA_ERR_UNSUPPORTED and
+ *     launches nothing.  CUDA errors at launch return MLA_ERR_CUDA.
+ *   - Conditions found on the device (a bounded wait that timed out, and with
+ *     device checks enabled, a block-table entry outside the cache) are written
+ *     to `device_status` when it is not NULL; the caller reads it after the
+ *     stream has completed.  No kernel traps or aborts.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned buffer */
+    MLA_ERR_UNSUPPORTED = 2,    /* a dimension this build does not implement */
+    MLA_ERR_CUDA = 3,           /* a CUDA runtime call failed */
+    MLA_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait gave up (device_status only) */
+    MLA_ERR_DEVICE_CHECK = 5    /* a device-side bounds check failed (device_status only) */
+} mla_status;
+
+#define MLA_HEAD_DIM_QK 576     /* 512 latent + 64 rope dims per row */
+#define MLA_HEAD_DIM_V 512      /* value = first 512 dims of the same row */
+#define MLA_PAGE_SIZE 64        /* tokens per cache page */
+#define MLA_MD_STRIDE 8         /* int32 per worker in tile_md */
+#define MLA_SPLIT_PIECE_COST 2  /* fixed cost of one piece, in pages (partition rule) */
+#define MLA_ROWS_PER_CTA 64     /* query rows (s_q * h_q, flattened) per decode CTA */
+
+/*
+ * mla_metadata_shape -- sizes for the split-KV metadata.
+ *
+ * num_workers: how many workers the decode grid uses on the current device:
+ *   max(1, SMs / ceil(s_q * h_q / 64)).  One worker is one CTA per 64-row block
+ *   of the query rows.  md_stride: MLA_MD_STRIDE.
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG (batch, h_q or s_q < 1, null outputs), or
+ * MLA_ERR_CUDA (no current device).
+ */
+int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_stride);
+
+/*
+ * mla_get_metadata -- the length-balanced split-KV tile scheduler.
+ *
+ * The pages ask for a kernel optimised for variable-length serving ("OpenSourceWeek
+ * Day 1: FlashMLA", opening paragraph; "DeepSeek merilis open source FlashMLA",
+ * release bullets) and give no partition rule.  The rule used here:
+ *   n_i = ceil(L_i / 64) pages; items_i = max(n_i, 1) (an empty sequence owns one
+ *   item so that its zero output is written); sequence i costs
+ *   MLA_SPLIT_PIECE_COST + items_i units, laid end to end from unit start_i, with
+ *   item j at unit start_i + MLA_SPLIT_PIECE_COST + j; cap = ceil(total / W);
+ *   the item at unit u goes to worker u / cap.
+ * Each worker thus owns a contiguous run of items.  A sequence whose items fall
+ * to k workers has k pieces (splits), merged by log-sum-exp in the decode call.
+ *
+ * cache_seqlens: device int32 [batch], each >= 0.
+ * tile_md:       device int32 [num_workers * 8], written:
+ *                [begin_seq, begin_item, end_seq, end_item (exclusive),
+ *                 begin_split (piece index of begin_seq within that sequence),
+ *                 num_pieces (0 = idle worker, then all fields are 0), 0, 0]
+ * num_splits:    device int32 [batch + 1], written: exclusive prefix sum of the
+ *                pieces per sequence (num_splits[0] = 0).
+ * num_workers:   >= 1; normally the value from mla_metadata_shape.  The same
+ *                value must be passed to mla_decode_kvcache.
+ * h_q, s_q:      checked only (> 0); the rule itself depends on lengths and W.
+ * One CTA; integer only; no host synchronisation.  batch <= 65536.
+ */
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int h_q, int s_q,
+                     int32_t* tile_md, int32_t* num_splits, int num_workers, void* stream);
+
+/*
+ * mla_workspace_size -- bytes of scratch mla_decode_kvcache needs for split
+ * partials: (batch + num_workers) pieces of s_q * h_q rows, each with dv fp32
+ * values plus one fp32 lse, rounded up to 256 bytes.  Returns 0 for invalid
+ * arguments.
+ */
+size_t mla_workspace_size(int batch, int s_q, int h_q, int dv, int num_workers);
+
+/*
+ * mla_decode_kvcache -- the decode itself.
+ *
+ * q:            device bf16 [batch, s_q, h_q, 576], 16-byte aligned.
+ * kcache:       device bf16 [num_blocks, 64, 576], 16-byte aligned.
+ * num_blocks:   pages in kcache (1 <= num_blocks, num_blocks * 64 < 2^31).
+ * block_table:  device int32 [batch, bt_stride]; entries [0, ceil(L_i/64)) of
+ *               row i name pages of kcache (the rest are never read).
+ * cache_seqlens: device int32 [batch], 0 <= L_i <= bt_stride * 64.
+ * d, dv:        must be 576 and 512 (MLA_ERR_UNSUPPORTED otherwise).
+ * softmax_scale: multiplies the dot products before the softmax.
+ * causal:       0 or 1, see the header comment.
+ * tile_md, num_splits, num_workers: from mla_get_metadata on the same
+ *               cache_seqlens (the same stream order makes them ready).
+ * workspace:    device scratch of at least mla_workspace_size(...) bytes,
+ *               256-byte aligned; contents need not be initialised.
+ * out:          device bf16 [batch, s_q, h_q, 512], written.
+ * lse:          device fp32 [batch, h_q, s_q], written (natural log).
+ * device_status: device int32, or NULL; receives MLA_ERR_DEVICE_* on a device
+ *               condition (never reset by the library: the caller zeroes it).
+ * Requires 1 <= s_q * h_q <= 65536 (MLA_ERR_UNSUPPORTED otherwise).
+ * Launches the decode kernel and, when a sequence has more than one piece,
+ * the split-combine kernel, on `stream`.
+ */
+int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
+                       const int32_t* block_table, int bt_stride,
+                       const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                       int d, int dv, float softmax_scale, int causal,
+                       const int32_t* tile_md, const int32_t* num_splits, int num_workers,
+                       void* workspace, size_t workspace_bytes,
+                       void* out, float* lse, int32_t* device_status, void* stream);
+
+/* mla_error_string -- static text for a status code (never NULL). */
+const char* mla_error_string(int status);
+
+/* mla_version -- build identification string (never NULL). */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

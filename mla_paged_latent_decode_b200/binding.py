@@ -1,0 +1,150 @@
+"""Python binding over the C ABI in include/mla_decode.h.
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every step of the decode runs in the library's kernels.  There is no
+fallback: if the compiled library is missing the import of this module fails,
+and on a machine without a CUDA device the compute calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+D_QK = 576
+D_V = 512
+PAGE = 64
+MD_STRIDE = 8
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_CUDA = 3
+MLA_ERR_DEVICE_TIMEOUT = 4
+MLA_ERR_DEVICE_CHECK = 5
+
+EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
+           "mla_error_string", "mla_version")
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {error_string(code)}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    path = os.environ.get("MLA_DECODE_LIB", _build.LIB_PATH)
+    if not os.path.exists(path):
+        raise ImportError(f"libmla_decode.so not built ({path}); run "
+                          "`python -m mla_paged_latent_decode_b200.build`")
+    lib = ctypes.CDLL(path)
+    p, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.mla_metadata_shape.argtypes = [i32, i32, i32, ip, ip]
+    lib.mla_metadata_shape.restype = i32
+    lib.mla_get_metadata.argtypes = [p, i32, i32, i32, p, p, i32, p]
+    lib.mla_get_metadata.restype = i32
+    lib.mla_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.mla_workspace_size.restype = sz
+    lib.mla_decode_kvcache.argtypes = [p, p, i64, p, i32, p, i32, i32, i32, i32, i32, f32, i32,
+                                       p, p, i32, p, sz, p, p, p, p]
+    lib.mla_decode_kvcache.restype = i32
+    lib.mla_error_string.argtypes = [i32]
+    lib.mla_error_string.restype = ctypes.c_char_p
+    lib.mla_version.argtypes = []
+    lib.mla_version.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+LIB_PATH = lib._name
+
+
+def error_string(code: int) -> str:
+    return lib.mla_error_string(int(code)).decode()
+
+
+def version() -> str:
+    return lib.mla_version().decode()
+
+
+def _check(code: int, what: str):
+    if code != MLA_OK:
+        raise MLAError(code, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def metadata_shape(batch: int, h_q: int, s_q: int) -> tuple[int, int]:
+    """(num_workers, md_stride) for the current CUDA device."""
+    nw, st = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.mla_metadata_shape(batch, h_q, s_q, ctypes.byref(nw), ctypes.byref(st)),
+           "mla_metadata_shape")
+    return nw.value, st.value
+
+
+def workspace_size(batch: int, s_q: int, h_q: int, num_workers: int, dv: int = D_V) -> int:
+    return int(lib.mla_workspace_size(batch, s_q, h_q, dv, num_workers))
+
+
+def get_mla_metadata(cache_seqlens: torch.Tensor, h_q: int, s_q: int,
+                     num_workers: int | None = None):
+    """Split-KV tile scheduler.  Returns (tile_md [W, 8] int32, num_splits [b + 1] int32),
+    both on cache_seqlens' device, produced on the current stream."""
+    assert cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32
+    assert cache_seqlens.dim() == 1 and cache_seqlens.is_contiguous()
+    dev = cache_seqlens.device
+    b = cache_seqlens.numel()
+    with torch.cuda.device(dev):
+        if num_workers is None:
+            num_workers, _ = metadata_shape(b, h_q, s_q)
+        tile_md = torch.empty((num_workers, MD_STRIDE), dtype=torch.int32, device=dev)
+        num_splits = torch.empty((b + 1,), dtype=torch.int32, device=dev)
+        _check(lib.mla_get_metadata(_ptr(cache_seqlens), b, h_q, s_q, _ptr(tile_md),
+                                    _ptr(num_splits), num_workers, _stream_handle(dev)),
+               "mla_get_metadata")
+    return tile_md, num_splits
+
+
+def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
+                       cache_seqlens: torch.Tensor, dv: int, tile_md: torch.Tensor,
+                       num_splits: torch.Tensor, softmax_scale: float, causal: bool = False,
+                       out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None,
+                       device_status: torch.Tensor | None = None):
+    """Paged MLA decode.  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q] fp32)."""
+    b, s_q, h_q, d = q.shape
+    dev = q.device
+    for t in (q, kcache, block_table, cache_seqlens, tile_md, num_splits):
+        assert t.is_cuda and t.device == dev and t.is_contiguous()
+    assert q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
+    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
+    assert kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d
+    assert block_table.dim() == 2 and block_table.shape[0] == b
+    num_workers = tile_md.shape[0]
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty((b, s_q, h_q, dv), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+        need = workspace_size(b, s_q, h_q, num_workers, dv)
+        if workspace is None:
+            workspace = torch.empty((max(need, 256),), dtype=torch.uint8, device=dev)
+        rc = lib.mla_decode_kvcache(
+            _ptr(q), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.shape[1],
+            _ptr(cache_seqlens), b, s_q, h_q, d, dv, float(softmax_scale), int(bool(causal)),
+            _ptr(tile_md), _ptr(num_splits), num_workers, _ptr(workspace), workspace.numel(),
+            _ptr(out), _ptr(lse), _ptr(device_status), _stream_handle(dev))
+        _check(rc, "mla_decode_kvcache")
+    return out, lse

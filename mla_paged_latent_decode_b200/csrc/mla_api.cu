@@ -1,0 +1,195 @@
+// mla_api.cu -- the extern "C" boundary declared in include/mla_decode.h.
+//
+// Host-side argument validation, TMA tensor-map construction (through the
+// driver entry point, so the library links only the static CUDA runtime), and
+// the launches of the scheduler, decode and combine kernels on the caller's
+// stream.  Nothing here allocates device memory or synchronises.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "mla_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int current_sm_count(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+  int v = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return MLA_ERR_CUDA;
+    g_sm_count[dev].store(v, std::memory_order_relaxed);
+  }
+  *sms = v;
+  return MLA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// A [rows, 576] bf16 row-major matrix read in 64 x 64 boxes with 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kDqk) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int row_blocks(int s_q, int h_q) {
+  const int rows = s_q * h_q;
+  return (rows + mla::kRowsPerCta - 1) / mla::kRowsPerCta;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_error_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK: success";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: invalid argument (null, size or alignment)";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: unsupported dimension";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: a device-side wait timed out";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: a device-side bounds check failed";
+    default: return "unknown mla status";
+  }
+}
+
+const char* mla_version(void) {
+  return "mla_paged_latent_decode_b200 sm_100a (tcgen05 M=64 decode, 2-stage TMA)";
+}
+
+int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_stride) {
+  if (batch < 1 || h_q < 1 || s_q < 1 || num_workers == nullptr || md_stride == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s_q) * h_q > 65536) return MLA_ERR_UNSUPPORTED;
+  int sms = 0;
+  int rc = current_sm_count(&sms);
+  if (rc != MLA_OK) return rc;
+  const int rb = row_blocks(s_q, h_q);
+  *num_workers = sms / rb > 1 ? sms / rb : 1;
+  *md_stride = MLA_MD_STRIDE;
+  return MLA_OK;
+}
+
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int h_q, int s_q,
+                     int32_t* tile_md, int32_t* num_splits, int num_workers, void* stream) {
+  if (cache_seqlens == nullptr || tile_md == nullptr || num_splits == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 65536 || h_q < 1 || s_q < 1 || num_workers < 1 ||
+      num_workers > (1 << 20))
+    return MLA_ERR_INVALID_ARG;
+  cudaError_t e = mla::launch_metadata(cache_seqlens, batch, num_workers, tile_md, num_splits,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+size_t mla_workspace_size(int batch, int s_q, int h_q, int dv, int num_workers) {
+  if (batch < 1 || s_q < 1 || h_q < 1 || dv != mla::kDv || num_workers < 1) return 0;
+  const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
+  const size_t rows = static_cast<size_t>(s_q) * static_cast<size_t>(h_q);
+  return round_up(slots * rows * dv * sizeof(float), 256) + round_up(slots * rows * sizeof(float), 256);
+}
+
+int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
+                       const int32_t* block_table, int bt_stride,
+                       const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                       int d, int dv, float softmax_scale, int causal,
+                       const int32_t* tile_md, const int32_t* num_splits, int num_workers,
+                       void* workspace, size_t workspace_bytes,
+                       void* out, float* lse, int32_t* device_status, void* stream) {
+  if (q == nullptr || kcache == nullptr || block_table == nullptr || cache_seqlens == nullptr ||
+      tile_md == nullptr || num_splits == nullptr || out == nullptr || lse == nullptr ||
+      workspace == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (d != mla::kDqk || dv != mla::kDv) return MLA_ERR_UNSUPPORTED;
+  if (batch < 1 || s_q < 1 || h_q < 1 || bt_stride < 1 || num_workers < 1 ||
+      num_workers > (1 << 20) || (causal != 0 && causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s_q) * h_q > 65536) return MLA_ERR_UNSUPPORTED;
+  if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * s_q * h_q >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+      !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_workspace_size(batch, s_q, h_q, dv, num_workers);
+  if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
+
+  const int rows = s_q * h_q;
+  CUtensorMap tm_q, tm_kv;
+  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
+  if (!make_row_map(&tm_kv, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage))
+    return MLA_ERR_CUDA;
+
+  const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             round_up(slots * rows * dv * sizeof(float), 256));
+
+  mla::DecodeParams p{};
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.status = device_status;
+  p.bt_stride = bt_stride;
+  p.num_blocks = num_blocks;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = rows;
+  p.causal = causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mla::launch_decode(tm_q, tm_kv, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
+
+  mla::CombineParams c{};
+  c.num_splits = num_splits;
+  c.part_o = part_o;
+  c.part_lse = part_lse;
+  c.out = static_cast<__nv_bfloat16*>(out);
+  c.lse = lse;
+  c.batch = batch;
+  c.s_q = s_q;
+  c.h_q = h_q;
+  c.rows = rows;
+  if (mla::launch_combine(c, st) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// mla_kernels.cuh -- parameter blocks and launch entry points shared by the
+// C-ABI layer (mla_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mla_decode.h"
+
+namespace mla {
+
+constexpr int kPage = MLA_PAGE_SIZE;      // tokens per page
+constexpr int kDqk = MLA_HEAD_DIM_QK;     // 576
+constexpr int kDv = MLA_HEAD_DIM_V;       // 512
+constexpr int kRowsPerCta = MLA_ROWS_PER_CTA;
+constexpr int kMdStride = MLA_MD_STRIDE;
+constexpr int kPieceCost = MLA_SPLIT_PIECE_COST;
+
+// Bounded device waits give up after this long (then report MLA_ERR_DEVICE_TIMEOUT).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct DecodeParams {
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  const int32_t* tile_md;
+  const int32_t* num_splits;
+  __nv_bfloat16* out;   // [b, s_q, h_q, 512]
+  float* lse;           // [b, h_q, s_q]
+  float* part_o;        // [pieces, rows, 512]
+  float* part_lse;      // [pieces, rows]
+  int32_t* status;      // nullable
+  int64_t bt_stride;
+  int64_t num_blocks;
+  int batch, s_q, h_q, rows;  // rows = s_q * h_q
+  int causal;
+  float scale_log2;     // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+  const int32_t* num_splits;
+  const float* part_o;
+  const float* part_lse;
+  __nv_bfloat16* out;
+  float* lse;
+  int batch, s_q, h_q, rows;
+};
+
+// Launchers (return cudaGetLastError() of their launch).
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int32_t* tile_md,
+                            int32_t* num_splits, cudaStream_t stream);
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
+                          const DecodeParams& p, int num_workers, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace mla

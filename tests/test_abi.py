@@ -1,0 +1,105 @@
+"""The C ABI library loads and exports what include/mla_decode.h declares (no GPU).
+
+Only host-side paths run here: status strings, sizes, and argument checks that
+return before any CUDA call.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from mla_paged_latent_decode_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla_decode.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(mla_[a-z_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_library_links_no_cuda_driver_or_torch():
+    out = subprocess.run(["readelf", "-d", binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    needed = re.findall(r"\(NEEDED\)\s+Shared library: \[(.+?)\]", out)
+    assert not any(n.startswith("libcuda.so") for n in needed)
+    assert not any("torch" in n for n in needed)
+
+
+def test_error_strings():
+    for code in range(6):
+        assert binding.error_string(code).startswith("MLA_")
+    assert "unknown" in binding.error_string(99)
+    assert "sm_100a" in binding.version()
+
+
+def test_workspace_size():
+    ws = binding.workspace_size(64, 1, 128, 74)
+    slots, rows = 64 + 74, 128
+    expect = -(-(slots * rows * 512 * 4) // 256) * 256 + -(-(slots * rows * 4) // 256) * 256
+    assert ws == expect
+    assert binding.lib.mla_workspace_size(0, 1, 128, 512, 74) == 0
+    assert binding.lib.mla_workspace_size(4, 1, 128, 256, 74) == 0
+
+
+def _decode_raw(**kw):
+    args = dict(q=1 << 12, kcache=1 << 12, num_blocks=4, block_table=1 << 12, bt_stride=3,
+                cache_seqlens=1 << 12, batch=2, s_q=1, h_q=16, d=576, dv=512, scale=0.07,
+                causal=0, tile_md=1 << 12, num_splits=1 << 12, num_workers=148,
+                workspace=1 << 12, workspace_bytes=1 << 30, out=1 << 12, lse=1 << 12)
+    args.update(kw)
+    v = ctypes.c_void_p
+    return binding.lib.mla_decode_kvcache(
+        v(args["q"]), v(args["kcache"]), args["num_blocks"], v(args["block_table"]),
+        args["bt_stride"], v(args["cache_seqlens"]), args["batch"], args["s_q"], args["h_q"],
+        args["d"], args["dv"], args["scale"], args["causal"], v(args["tile_md"]),
+        v(args["num_splits"]), args["num_workers"], v(args["workspace"]),
+        args["workspace_bytes"], v(args["out"]), v(args["lse"]), v(0), v(0))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(out=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(d=512), binding.MLA_ERR_UNSUPPORTED),
+    (dict(dv=576), binding.MLA_ERR_UNSUPPORTED),
+    (dict(batch=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(causal=2), binding.MLA_ERR_INVALID_ARG),
+    (dict(num_workers=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(num_blocks=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(num_blocks=1 << 25), binding.MLA_ERR_INVALID_ARG),
+    (dict(q=(1 << 12) + 2), binding.MLA_ERR_INVALID_ARG),
+    (dict(workspace=(1 << 12) + 16), binding.MLA_ERR_INVALID_ARG),
+    (dict(workspace_bytes=100), binding.MLA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.MLA_ERR_INVALID_ARG),
+    (dict(s_q=512, h_q=256), binding.MLA_ERR_UNSUPPORTED),
+])
+def test_decode_host_validation(kw, code):
+    # every case fails validation before any CUDA call, so no device is needed
+    assert _decode_raw(**kw) == code
+
+
+def test_metadata_host_validation():
+    v = ctypes.c_void_p
+    assert binding.lib.mla_get_metadata(v(0), 2, 16, 1, v(4096), v(4096), 148, v(0)) == 1
+    assert binding.lib.mla_get_metadata(v(4096), 0, 16, 1, v(4096), v(4096), 148, v(0)) == 1
+    assert binding.lib.mla_get_metadata(v(4096), 2, 16, 1, v(4096), v(4096), 0, v(0)) == 1
+    nw, st = ctypes.c_int(0), ctypes.c_int(0)
+    assert binding.lib.mla_metadata_shape(0, 16, 1, ctypes.byref(nw), ctypes.byref(st)) == 1

@@ -1,0 +1,149 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerance of the decode: |out - ref| <= 1e-2 + 1e-2 |ref| on the bf16 output,
+|lse - ref| <= 1e-3, and the split metadata bit-exact against the CPU
+restatement of the partition rule.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mla_paged_latent_decode_b200 import synth
+from parity import (check_metadata, full_parity, run_cuda, sampled_parity, assert_close_out,
+                    assert_close_lse, expected_workers)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_workload(cuda_device):
+    inp = synth.make_inputs("tiny", seed=0)
+    full_parity(inp, cuda_device)
+
+
+@pytest.mark.parametrize("h_q", [1, 16, 64, 128])
+@pytest.mark.parametrize("s_q,causal", [(1, False), (2, True), (2, False)])
+def test_small_shapes(cuda_device, h_q, s_q, causal):
+    # several pages, ragged tails, one sequence shorter than a page
+    w = synth.custom_workload(4, s_q, h_q, [1, 63, 130, 257], causal=causal)
+    inp = synth.make_inputs(w, seed=100 + h_q + s_q)
+    full_parity(inp, cuda_device)
+
+
+@pytest.mark.parametrize("num_workers", [1, 3, 17, 148, 600])
+def test_forced_splits(cuda_device, num_workers):
+    # num_workers controls how finely sequences are cut: 1 = no splits at all,
+    # 600 = a piece per page; every plan must give the same answer
+    w = synth.custom_workload(3, 2, 32, [700, 5, 1100], causal=True)
+    inp = synth.make_inputs(w, seed=7)
+    full_parity(inp, cuda_device, num_workers=num_workers)
+
+
+def test_empty_and_degenerate_sequences(cuda_device):
+    # L = 0 (nothing visible), L = 1 < s_q (first query empty under causal), exact pages
+    w = synth.custom_workload(5, 2, 16, [0, 1, 64, 128, 2], causal=True)
+    inp = synth.make_inputs(w, seed=3)
+    res, ref_out, ref_lse = full_parity(inp, cuda_device)
+    assert np.all(res["out"][0] == 0) and np.all(np.isneginf(res["lse"][0]))
+    assert np.all(res["out"][1, 0] == 0) and np.all(np.isneginf(res["lse"][1, :, 0]))
+
+
+def test_poisoned_tails_and_pad_pages(cuda_device):
+    w = synth.custom_workload(4, 2, 128, [37, 130, 64, 300], causal=True)
+    inp = synth.make_inputs(w, seed=5, poison=True)
+    full_parity(inp, cuda_device)
+    full_parity(inp, cuda_device, num_workers=50)
+
+
+def test_page_permutation_bit_exact(cuda_device):
+    w = synth.custom_workload(3, 1, 128, [500, 64, 1000])
+    inp = synth.make_inputs(w, seed=9)
+    a = run_cuda(inp, cuda_device)
+    nb = inp.kcache.shape[0]
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(1))
+    moved = torch.empty_like(inp.kcache)
+    moved[perm] = inp.kcache
+    inp.kcache = moved
+    inp.block_table = perm[inp.block_table.long()].to(torch.int32)
+    b = run_cuda(inp, cuda_device)
+    np.testing.assert_array_equal(a["out"], b["out"])
+    np.testing.assert_array_equal(a["lse"], b["lse"])
+
+
+def test_dominant_key_and_large_logits(cuda_device):
+    # a key whose logit dominates by ~74 must be selected exactly; logits far
+    # above the rescale threshold exercise the running-max correction
+    L = 4000
+    w = synth.custom_workload(2, 1, 64, [L, L])
+    inp = synth.make_inputs(w, seed=11)
+    inp.q[..., 575] = 1.0
+    inp.kcache[..., 575] = 0.0
+    for i, t_star in enumerate([3900, 17]):
+        page = int(inp.block_table[i, t_star // 64])
+        inp.kcache[page, t_star % 64, 575] = 1024.0
+    # growing logits along the sequence force repeated rescales
+    for t in range(0, L, 64):
+        page = int(inp.block_table[1, t // 64])
+        inp.kcache[page, :, 574] = float(t) / 16.0
+    inp.q[1, :, :, 574] = 1.0
+    full_parity(inp, cuda_device)
+
+
+@pytest.mark.parametrize("name", ["dsv3_decode", "varlen_h16", "spec_causal", "skewed_long"])
+def test_full_size_workloads_sampled(cuda_device, name):
+    inp = synth.make_inputs(name, seed=0)
+    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
+    extra = [(0, 0, 0), (b - 1, s_q - 1, h_q - 1)]
+    sampled_parity(inp, cuda_device, n_rows=48, extra_rows=extra)
+
+
+def test_default_workers_match_formula(cuda_device):
+    from mla_paged_latent_decode_b200 import binding
+    for s_q, h_q in [(1, 16), (1, 128), (2, 128), (1, 1), (4, 128)]:
+        nw, stride = binding.metadata_shape(8, h_q, s_q)
+        assert stride == 8
+        assert nw == expected_workers(cuda_device, s_q, h_q)
+
+
+def test_metadata_bit_exact_many_shapes(cuda_device):
+    from mla_paged_latent_decode_b200 import binding
+    g = torch.Generator().manual_seed(0)
+    for b in (1, 2, 7, 128, 1000, 3000):
+        lens = torch.randint(0, 20000, (b,), generator=g, dtype=torch.int32)
+        lens[::5] = 0
+        sl = lens.to(cuda_device)
+        for W in (1, 5, 74, 148, 2000):
+            tile_md, num_splits = binding.get_mla_metadata(sl, 16, 1, W)
+            torch.cuda.synchronize()
+            res = {"tile_md": tile_md.cpu(), "num_splits": num_splits.cpu()}
+
+            class _I:
+                cache_seqlens = lens
+            check_metadata(_I, res, W)
+
+
+def test_host_validation_rejects_bad_arguments(cuda_device):
+    from mla_paged_latent_decode_b200 import binding
+    inp = synth.make_inputs("tiny", seed=0)
+    q = inp.q.to(cuda_device)
+    kc = inp.kcache.to(cuda_device)
+    bt = inp.block_table.to(cuda_device)
+    sl = inp.cache_seqlens.to(cuda_device)
+    md, ns = binding.get_mla_metadata(sl, inp.h_q, inp.s_q)
+    with pytest.raises(binding.MLAError) as e:
+        binding.mla_decode_kvcache(q, kc, bt, sl, 256, md, ns, inp.scale)
+    assert e.value.code == binding.MLA_ERR_UNSUPPORTED
+    small_ws = torch.empty(16, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(binding.MLAError) as e:
+        binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, workspace=small_ws)
+    assert e.value.code == binding.MLA_ERR_INVALID_ARG
+
+
+def test_overlong_sequence_is_reported_not_read(cuda_device):
+    # a length beyond the block-table row is flagged on the device; the kernel
+    # reads no entry past the row
+    w = synth.custom_workload(2, 1, 16, [100, 64])
+    inp = synth.make_inputs(w, seed=2)
+    inp.cache_seqlens[1] = 64 * inp.block_table.shape[1] + 50
+    res = run_cuda(inp, cuda_device)
+    from mla_paged_latent_decode_b200 import binding
+    assert res["status"] == binding.MLA_ERR_DEVICE_CHECK
