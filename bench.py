@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the paged MLA decode on B200: TB/s, TFLOPS and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload dsv3_decode]
+
+A step is one pass of the whole hot path over one batch: the split-KV
+scheduler, the decode kernel and (for split sequences) the combine kernel, all
+through the C ABI.  The default workload is DeepSeek-V3-shaped decode: batch
+64, s_q 1, 128 heads, every sequence 4096 tokens, 64-token pages shuffled in
+the block table, q and cache ~ N(0, 1) in bf16, scale 1/sqrt(192).
+
+Timing: W untimed warm-up steps, then exactly K steps, each preceded by a
+256 MB device write that flushes L2 (outside the step's event pair); every
+step is timed with CUDA events on the launching stream; the K timed steps are
+bracketed by a barrier and a device synchronise on both sides; the reported
+time is the maximum over ranks.  With N > 1 every rank runs the same workload
+on its own GPU (independent replicas; the decode has no cross-GPU exchange).
+
+`--impl reference` times the fp64 CPU oracle on this host instead (bounded
+samples of the same workload), printing the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_paged_latent_decode_b200 import synth  # noqa: E402
+
+METRIC = "MLA decode TB/s and TFLOPS on one B200 (bf16, paged KV), % of roofline"
+UNIT = "TB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dsv3_decode_traffic.md")
+DECODE_SRC = os.path.join(ROOT, "mla_paged_latent_decode_b200", "csrc", "mla_decode_sm100.cu")
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def decode_source_sha():
+    with open(DECODE_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current decode kernel source and this workload; else None."""
+    if workload != "dsv3_decode" or not os.path.exists(TRAFFIC_FILE):
+        return None
+    fields = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("decode_kernel_source_sha256_16") != decode_source_sha():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self._nvml = pynvml
+            self._handle = None
+            for k in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(k)
+                hu = pynvml.nvmlDeviceGetUUID(h)
+                hu = hu.decode() if isinstance(hu, bytes) else hu
+                if str(uuid) in hu or hu.endswith(str(uuid)):
+                    self._handle = h
+            if self._handle is None:
+                self._handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._handle = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                mask = get(self._handle)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._handle is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def workload_config(inp, extra=None):
+    w = inp.workload
+    cfg = {"workload": f"{w.name}: {w.description}", "batch": inp.batch, "s_q": inp.s_q,
+           "h_q": inp.h_q, "d_qk": 576, "dv": 512, "page": 64,
+           "total_cached_tokens": int(inp.cache_seqlens.sum()), "causal": bool(inp.causal),
+           "scale": inp.scale, "seed": inp.seed,
+           "l2": "flushed before every timed step by a 256 MB device write"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample(inp, target_s: float):
+    """Pick a sample of the workload that the fp64 oracle finishes in about
+    target_s: first more heads of one sequence, then more whole sequences.
+    Returns (sample inputs, seconds of the last trial, description)."""
+    import oracle
+    b, h_q = inp.batch, inp.h_q
+    n_seq, n_head = 1, 1
+    while True:
+        sub = subset(inp, n_seq, n_head)
+        t0 = time.perf_counter()
+        oracle.decode(sub.q, sub.kcache, sub.block_table, sub.cache_seqlens, sub.scale, sub.causal)
+        dt = time.perf_counter() - t0
+        done = n_seq >= b and n_head >= h_q
+        if dt >= target_s or done:
+            what = (f"{n_seq} of {b} sequences x {n_head} of {h_q} heads "
+                    f"(all query positions), fp64 C oracle")
+            return sub, dt, what
+        grow = max(2.0, 0.9 * target_s / max(dt, 1e-4))
+        if n_head < h_q:
+            n_head = min(h_q, int(n_head * grow))
+        else:
+            n_seq = min(b, int(n_seq * grow))
+
+
+def subset(inp, n_seq, n_head=None):
+    """The first n_seq sequences (and first n_head heads) of a workload."""
+    import copy
+    sub = copy.copy(inp)
+    n_head = inp.h_q if n_head is None else n_head
+    sub.q = inp.q[:n_seq, :, :n_head].contiguous()
+    sub.block_table = inp.block_table[:n_seq].contiguous()
+    sub.cache_seqlens = inp.cache_seqlens[:n_seq].contiguous()
+    return sub
+
+
+def oracle_rate(sub, seconds):
+    nbytes, flops = synth.algorithmic_work(sub)
+    return nbytes / seconds / 1e12, flops / seconds / 1e12
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}; launch with torchrun")
+    return rank, local, world
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    """The oracle arm: rank 0 only, on this host's cores."""
+    if rank != 0:
+        return None
+    import oracle
+    inp = synth.make_inputs(args.workload, seed=0)
+    # size the per-step sample once so that all steps together take about two minutes
+    per_step_target = max(0.01, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    sub, _, sample = oracle_sample(inp, per_step_target)
+    threads = oracle.threads()
+    for _ in range(args.warmup):
+        oracle.decode(sub.q, sub.kcache, sub.block_table, sub.cache_seqlens, sub.scale, sub.causal)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode(sub.q, sub.kcache, sub.block_table, sub.cache_seqlens, sub.scale, sub.causal)
+        times.append(time.perf_counter() - t0)
+    nbytes, flops = synth.algorithmic_work(sub)
+    total = sum(times)
+    value = nbytes * args.steps / total / 1e12
+    sample = f"per step: {sample}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 inputs widened exactly to fp64)",
+        "config": workload_config(inp, {"sample": sample}),
+        "tflops": flops * args.steps / total / 1e12,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def run_cuda(args, rank, local, world):
+    from mla_paged_latent_decode_b200 import binding
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(args.workload, seed=0)
+    nbytes, flops = synth.algorithmic_work(inp)
+    q = inp.q.to(dev)
+    kc = inp.kcache.to(dev)
+    bt = inp.block_table.to(dev)
+    sl = inp.cache_seqlens.to(dev)
+    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
+    num_workers, _ = binding.metadata_shape(b, h_q, s_q)
+    out = torch.empty((b, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    ws = torch.empty((binding.workspace_size(b, s_q, h_q, num_workers),), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        md, ns = binding.get_mla_metadata(sl, h_q, s_q, num_workers)
+        ev_mid.record(stream)
+        binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal, out=out,
+                                   lse=lse, workspace=ws, device_status=status)
+
+    for _ in range(args.warmup):
+        ev_mid = torch.cuda.Event(enable_timing=True)
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_wall0 = time.perf_counter()
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            e0, ev_mid, e1 = events[k]
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall0
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    step_ms = [e0.elapsed_time(e1) for e0, _, e1 in events]
+    decode_ms = [m.elapsed_time(e1) for _, m, e1 in events]
+    meta_ms = [e0.elapsed_time(m) for e0, m, _ in events]
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during timing")
+
+    total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
+    all_bytes = reduce_sum(float(nbytes * args.steps), world, dev)
+    all_flops = reduce_sum(float(flops * args.steps), world, dev)
+    decode_avg_s = reduce_max(sum(decode_ms) / len(decode_ms) / 1e3, world, dev)
+
+    # end to end through the public API: per-step inputs copied in from pinned host
+    # memory and the outputs copied back, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq = inp.q.pin_memory()
+        hbt = inp.block_table.pin_memory()
+        hsl = inp.cache_seqlens.pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq, dbt, dsl = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dbt.copy_(hbt, non_blocking=True)
+            dsl.copy_(hsl, non_blocking=True)
+            md, ns = binding.get_mla_metadata(dsl, h_q, s_q, num_workers)
+            o, l = binding.mla_decode_kvcache(dq, kc, dbt, dsl, 512, md, ns, inp.scale,
+                                              inp.causal, out=out, lse=lse, workspace=ws)
+            hout.copy_(o, non_blocking=True)
+            hlse.copy_(l, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 200))
+        e2e_ms = []
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        for k in range(n_e2e):
+            flush.fill_(k & 0xFF)
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            z.record(stream)
+            e2e_ms.append((a, z))
+        torch.cuda.synchronize(dev)
+        e2e_total = reduce_max(sum(a.elapsed_time(z) for a, z in e2e_ms) / 1e3, world, dev)
+        e2e_bytes = reduce_sum(float(nbytes * n_e2e), world, dev)
+        h2d = hq.numel() * hq.element_size() + hbt.numel() * 4 + hsl.numel() * 4
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+        e2e = {"value": e2e_bytes / e2e_total / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "note": "q, block_table and cache_seqlens copied in, out and lse copied back each "
+                       "step; the latent cache stays resident in HBM as in serving"}
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    ms_per_step = total_s / args.steps * 1e3
+    value = all_bytes / total_s / 1e12
+    tflops = all_flops / total_s / 1e12
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        achieved = nbytes / decode_avg_s / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = flops / decode_avg_s / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q and latent cache, shuffled 64-token pages)",
+        "config": workload_config(inp, {"parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                                        "num_workers": num_workers}),
+        "tflops": tflops,
+        "roofline_frac": max(t_hbm, t_tc) / (ms_per_step / 1e3),
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                     "kernel": "mla_decode_kvcache call (decode kernel + split combine)",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s / 1.59 PFLOP/s"},
+        "kernel_us": {"metadata": statistics.median(meta_ms) * 1e3,
+                      "decode_call": statistics.median(decode_ms) * 1e3,
+                      "step": statistics.median(step_ms) * 1e3},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        sub, dt, what = oracle_sample(inp, args.cpu_seconds)
+        tbs, tfl = oracle_rate(sub, dt)
+        line["cpu_baseline"] = {
+            "value": tbs, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{what}, {dt:.1f} s", "tflops": tfl}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="dsv3_decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="approximate oracle time for the cpu_baseline sample")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "cuda":
+        raise SystemExit("--warmup must be at least 3")
+    rank, local, world = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_cuda(args, rank, local, world)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
