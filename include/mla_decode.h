@@ -49,7 +49,8 @@ typedef enum {
     MLA_ERR_UNSUPPORTED = 2,    /* a dimension this build does not implement */
     MLA_ERR_CUDA = 3,           /* a CUDA runtime call failed */
     MLA_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait gave up (device_status only) */
-    MLA_ERR_DEVICE_CHECK = 5    /* a device-side bounds check failed (device_status only) */
+    MLA_ERR_DEVICE_CHECK = 5,   /* a device-side bounds check failed (device_status only) */
+    MLA_ERR_SCRATCH_LIMIT = 6   /* workspace would exceed MLA_STATIC_SCRATCH_BYTES */
 } mla_status;
 
 #define MLA_HEAD_DIM_QK 576     /* 512 latent + 64 rope dims per row */
@@ -58,6 +59,7 @@ typedef enum {
 #define MLA_MD_STRIDE 8         /* int32 per worker in tile_md */
 #define MLA_SPLIT_PIECE_COST 2  /* fixed cost of one piece, in pages (partition rule) */
 #define MLA_ROWS_PER_CTA 64     /* query rows (s_q * h_q, flattened) per decode CTA */
+#define MLA_STATIC_SCRATCH_BYTES ((size_t)48 << 20) /* see mla_decode_kvcache_static_scratch */
 
 /*
  * mla_metadata_shape -- sizes for the split-KV metadata.
@@ -138,6 +140,39 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
                        const int32_t* tile_md, const int32_t* num_splits, int num_workers,
                        void* workspace, size_t workspace_bytes,
                        void* out, float* lse, int32_t* device_status, void* stream);
+
+/*
+ * mla_decode_kvcache_static_scratch -- mla_decode_kvcache for callers that
+ * cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for library
+ * users.  mla_decode_kvcache needs a workspace for the fp32 partial results of
+ * sequences split across workers.  Some callers cannot provide one, because
+ * they cannot call cudaMalloc: an engine that reserves all device memory up
+ * front in its own arena and allows no further allocation, or a
+ * latency-critical loop that must not allocate or free (cudaFree synchronises
+ * the device).  This call takes the same arguments minus the workspace and
+ * uses a fixed array of MLA_STATIC_SCRATCH_BYTES (48 MiB) compiled into the
+ * library instead; it calls no allocating routine.
+ *
+ * Limit: if mla_workspace_size(batch, s_q, h_q, dv, num_workers) exceeds
+ * MLA_STATIC_SCRATCH_BYTES it returns MLA_ERR_SCRATCH_LIMIT and launches
+ * nothing (fewer workers need less workspace).
+ * Every GPU that loads this part of the library holds the 48 MiB array until
+ * the process exits.  All calls on a device share it and it keeps the last
+ * call's contents (nothing in it needs to start at zero); calls that overlap
+ * on the GPU race on it, so serialise them.  The first call on each device
+ * looks up the array's device address; make that first call before any
+ * stream capture.  Otherwise identical to mla_decode_kvcache, including its
+ * errors.
+ */
+int mla_decode_kvcache_static_scratch(const void* q, const void* kcache, int64_t num_blocks,
+                                      const int32_t* block_table, int bt_stride,
+                                      const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                                      int d, int dv, float softmax_scale, int causal,
+                                      const int32_t* tile_md, const int32_t* num_splits,
+                                      int num_workers, void* out, float* lse,
+                                      int32_t* device_status, void* stream);
 
 /* mla_error_string -- static text for a status code (never NULL). */
 const char* mla_error_string(int status);

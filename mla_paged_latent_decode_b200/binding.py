@@ -25,9 +25,11 @@ MLA_ERR_UNSUPPORTED = 2
 MLA_ERR_CUDA = 3
 MLA_ERR_DEVICE_TIMEOUT = 4
 MLA_ERR_DEVICE_CHECK = 5
+MLA_ERR_SCRATCH_LIMIT = 6
+STATIC_SCRATCH_BYTES = 48 << 20
 
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-           "mla_error_string", "mla_version")
+           "mla_decode_kvcache_static_scratch", "mla_error_string", "mla_version")
 
 
 class MLAError(RuntimeError):
@@ -54,6 +56,9 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache.argtypes = [p, p, i64, p, i32, p, i32, i32, i32, i32, i32, f32, i32,
                                        p, p, i32, p, sz, p, p, p, p]
     lib.mla_decode_kvcache.restype = i32
+    lib.mla_decode_kvcache_static_scratch.argtypes = [p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
+                                                      f32, i32, p, p, i32, p, p, p, p]
+    lib.mla_decode_kvcache_static_scratch.restype = i32
     lib.mla_error_string.argtypes = [i32]
     lib.mla_error_string.restype = ctypes.c_char_p
     lib.mla_version.argtypes = []

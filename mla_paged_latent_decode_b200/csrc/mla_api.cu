@@ -80,6 +80,9 @@ const char* mla_error_string(int status) {
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
     case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: a device-side wait timed out";
     case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: a device-side bounds check failed";
+    case MLA_ERR_SCRATCH_LIMIT:
+      return "MLA_ERR_SCRATCH_LIMIT: workspace needed exceeds the library's static scratch "
+             "(MLA_STATIC_SCRATCH_BYTES)";
     default: return "unknown mla status";
   }
 }
