@@ -88,7 +88,7 @@ const char* mla_error_string(int status) {
 }
 
 const char* mla_version(void) {
-  return "mla_paged_latent_decode_b200 sm_100a (tcgen05 M=64 decode, 2-stage TMA)";
+  return "mla_paged_latent_decode_b200 sm_100a (tcgen05 M=64 decode, Q in TMEM, 3-stage TMA)";
 }
 
 int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_stride) {

@@ -1,32 +1,43 @@
 // mla_decode_sm100.cu -- MLA decode over a paged latent cache on sm_100a.
 //
 // One CTA owns one 64-row block of the flattened (s_q, h_q) query rows of one
-// worker's run of (sequence, page) items (see mla_metadata.cu).  Per page:
+// worker's run of (sequence, page) items (see mla_metadata.cu).
 //
-//   TMA   : the 64 x 576 bf16 page (72 KB) -> shared memory, 9 boxes of 64 x 64
-//           with 128-byte swizzle, through the block table; two stages.
-//   MMA   : S  = Q . K^T     tcgen05 M=64 N=64  K=576, A=Q (smem), B=page (smem)
-//           O += P . V       tcgen05 M=64 N=256 K=64 (x2 halves of dv=512),
-//                            A=P (smem), B=the same page tile read MN-major:
-//                            the value is dims 0..511 of the row already in
-//                            shared memory, so each page leaves HBM once.
-//   softmax warps: online softmax on S read from TMEM, P (bf16) -> shared
-//           memory, O rescaled in TMEM when the running max grows.
+// Data movement and math per page:
+//   TMA   : the 64 x 576 bf16 page (72 KB) -> shared memory as 9 boxes of
+//           64 x 64 with 128-byte swizzle, through the block table; a ring of
+//           three stages.  At the start of each piece the same ring also
+//           carries the piece's 64 query rows (72 KB), which the softmax warps
+//           move into tensor memory.
+//   MMA   : S  = Q . K^T    tcgen05 M=64 N=64 K=576, A = Q in TMEM, B = page
+//           O += P . V      tcgen05 M=64 N=256 K=64 (two halves of dv = 512),
+//                           A = P in SMEM, B = the same page tile read MN-major:
+//                           the value is dims 0..511 of the rows already in
+//                           shared memory, so each page leaves HBM once.
+//           S is double-buffered: QK^T of page j+1 runs while the softmax of
+//           page j does, and PV of page j follows.
+//   softmax warps: online softmax on S read from TMEM, P (bf16) -> SMEM, O
+//           rescaled in TMEM only when the running maximum grows past a
+//           threshold.
 //   epilogue: O / l -> bf16 out and lse, or fp32 partials for split sequences.
 //
-// TMEM (512 columns x 128 lanes): an M=64 accumulator occupies lanes 0-15 of
-// each 32-lane quarter.  O (64 x 512 fp32) takes all 512 columns of those
-// lanes; S (64 x 64 fp32) sits in the other half of each quarter (lane offset
-// 16), columns 0..63.  Thread t of softmax warp w therefore sees O row
-// 16w + t (t < 16) or S row 16w + t - 16 (t >= 16) in its lane.
+// Tensor memory (512 columns x 128 lanes).  An M=64 operand or accumulator
+// occupies 16 lanes of each 32-lane quarter; row r of a block lives in quarter
+// r / 16.  Lanes 0-15 of each quarter hold Q (columns 0..287, two bf16 per
+// column) and the two S buffers (columns 320..383, 384..447): the A operand and
+// the accumulator of QK^T must share lanes.  Lanes 16-31 hold O (columns
+// 0..511).  Softmax, rescale and epilogue use 16-lane TMEM accesses, so they
+// never touch lanes an MMA in flight is writing.
 //
 // Warp roles (192 threads): warps 0-3 softmax/correction/epilogue, warp 4 TMA
 // producer, warp 5 MMA issuer (and TMEM allocator).
 //
-// The method is "FlashMLA: Revolutionizing Efficient Decoding...", sections
-// 4.2.1-4.2.3 (TMA prefetch of 64-row latent blocks into shared memory, tensor
-// cores for QK^T and PV, softmax fused into the kernel) re-designed for the
-// 5th-generation tensor core: accumulators live in TMEM instead of registers.
+// The method follows "FlashMLA: Revolutionizing Efficient Decoding...",
+// sections 4.2.1-4.2.3 (TMA prefetch of 64-row latent blocks into shared
+// memory, tensor cores for QK^T and PV, softmax fused into the kernel),
+// re-designed for the 5th-generation tensor core: operands and accumulators
+// live in tensor memory, MMAs are issued by one thread, and the softmax runs in
+// warps of its own.
 #include "mla_kernels.cuh"
 #include "sm100_ptx.cuh"
 
@@ -34,32 +45,44 @@ namespace mla {
 namespace {
 
 constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kChunkBytes = 64 * 128;              // 64 rows x 64 bf16 (one swizzle column block)
 constexpr int kChunks = kDqk / 64;                 // 9
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 73728 = 64 x 576 bf16
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kPBytes = 64 * 128;                  // P: 64 rows x 64 tokens bf16
 
-constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kTileBytes;
+constexpr int kOffKV = 0;
 constexpr int kOffP = kOffKV + kStages * kTileBytes;
 constexpr int kOffBar = kOffP + kPBytes;
-enum Bar { kFull0 = 0, kEmpty0 = kStages, kQFull = 2 * kStages, kQEmpty, kSFull, kPFull, kOFull,
-           kOFree, kNumBars };
+enum Bar {
+  kFull0 = 0,
+  kEmpty0 = kStages,
+  kQFull = 2 * kStages,
+  kSFull0,
+  kSFull1,
+  kPFull,
+  kPvDone,
+  kOFull,
+  kNumBars
+};
 constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem address + abort flag
 constexpr int kSmemUsed = kOffMisc + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;       // slack to align the base to 1024 B
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 16u << 16;             // lane offset 16, column 0
+constexpr uint32_t kTmemQ = 0;                     // lanes 0-15, columns 0..287
+constexpr uint32_t kTmemS = 320;                   // lanes 0-15, S buffer b at 320 + 64 b
+constexpr uint32_t kTmemO = 16u << 16;             // lanes 16-31, columns 0..511
 constexpr float kRescaleThreshold = 8.0f;          // log2 units: P <= 2^8 before a rescale
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kTmemS + 128 <= kTmemCols, "tensor memory budget");
 
 struct Piece {
   int seq, pg0, npg, split_idx;
@@ -88,13 +111,19 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Bounded wait whose outcome is the same for every lane of the warp, so that
+// warp-collective TMEM accesses that follow are reached by all lanes or none.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort, kWaitLimitNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sq = smem + kOffQ;
   uint8_t* skv = smem + kOffKV;
   uint8_t* sp = smem + kOffP;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -116,12 +145,12 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bar[kFull0 + s], 1);
       mbar_init(&bar[kEmpty0 + s], 1);
     }
-    mbar_init(&bar[kQFull], 1);
-    mbar_init(&bar[kQEmpty], 1);
-    mbar_init(&bar[kSFull], 1);
-    mbar_init(&bar[kPFull], 128);
+    mbar_init(&bar[kQFull], kSoftmaxThreads);
+    mbar_init(&bar[kSFull0], 1);
+    mbar_init(&bar[kSFull1], 1);
+    mbar_init(&bar[kPFull], kSoftmaxThreads);
+    mbar_init(&bar[kPvDone], 1);
     mbar_init(&bar[kOFull], 1);
-    mbar_init(&bar[kOFree], 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -134,241 +163,311 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // The stage ring carries, per piece with pages, one entry for the query rows
+  // followed by one entry per page; every role counts entries the same way.
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_kv);
-      int q_loads = 0, kv_loads = 0;
+      int entries = 0;
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (p.seqlens[pz.seq] > p.bt_stride * kPage) report(p.status, MLA_ERR_DEVICE_CHECK);
         if (pz.npg == 0) continue;
-        if (q_loads > 0) ok = mbar_wait(&bar[kQEmpty], (q_loads - 1) & 1, abort_flag, kWaitLimitNs);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar[kQFull], kTileBytes);
-        const int qrow = pz.seq * p.rows + rb * kRowsPerCta;
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_2d(sq + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kQFull]);
-        ++q_loads;
         const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
-        for (int j = 0; j < pz.npg; ++j) {
-          const int stage = kv_loads % kStages, use = kv_loads / kStages;
+        for (int e = -1; e < pz.npg; ++e) {  // e = -1: the query rows
+          const int stage = entries % kStages, use = entries / kStages;
           if (use > 0) {
             ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, kWaitLimitNs);
             if (!ok) break;
           }
-          const int page = __ldg(bt + pz.pg0 + j);
-          mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
           uint8_t* dst = skv + stage * kTileBytes;
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_2d(dst + c * kChunkBytes, &tm_kv, c * 64, page * kPage, &bar[kFull0 + stage]);
-          ++kv_loads;
+          mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
+          if (e < 0) {
+            const int qrow = pz.seq * p.rows + rb * kRowsPerCta;
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
+          } else {
+            const int page = __ldg(bt + pz.pg0 + e);
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_kv, c * 64, page * kPage,
+                          &bar[kFull0 + stage]);
+          }
+          ++entries;
         }
       }
       // Before leaving, let every copy this thread issued land (bounded).
-      for (int s = 0; s < kStages && s < kv_loads; ++s) {
-        const int n = kv_loads - 1 - s;  // the last load issued into some stage
+      for (int s = 0; s < kStages && s < entries; ++s) {
+        const int n = entries - 1 - s;
         mbar_wait(&bar[kFull0 + n % kStages], (n / kStages) & 1, abort_flag, kWaitLimitNs);
       }
-      if (q_loads > 0) mbar_wait(&bar[kQFull], (q_loads - 1) & 1, abort_flag, kWaitLimitNs);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int q_uses = 0, kv_uses = 0, p_uses = 0, pieces_done = 0;
+      int entries = 0, pages = 0, qloads = 0;
       bool ok = true;
-      const uint32_t q_base = smem_addr(sq), kv_base = smem_addr(skv), p_base = smem_addr(sp);
+      const uint32_t kv_base = smem_addr(skv), p_base = smem_addr(sp);
+      auto issue_qk = [&](int entry, int page_index) -> bool {
+        const int stage = entry % kStages;
+        if (!mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, kWaitLimitNs))
+          return false;
+        tc_fence_after();
+        const uint32_t tile = kv_base + stage * kTileBytes;
+        const uint32_t d = tmem + kTmemS + 64 * (page_index & 1);
+        const uint64_t b0 = smem_desc_sw128(tile, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kDqk / 16; ++kk) {
+          // K-step kk: swizzle block kk/4, 32-byte step (kk%4) inside it
+          const uint32_t boff = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_ts(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar[kSFull0 + (page_index & 1)]);
+        return true;
+      };
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (pz.npg == 0) continue;
-        ok = mbar_wait(&bar[kQFull], q_uses & 1, abort_flag, kWaitLimitNs);
-        ++q_uses;
-        if (ok && pieces_done > 0)
-          ok = mbar_wait(&bar[kOFree], (pieces_done - 1) & 1, abort_flag, kWaitLimitNs);
+        const int q_entry = entries;   // copied into TMEM by the softmax warps
+        const int first = entries + 1;
+        entries += 1 + pz.npg;
+        ok = mbar_wait(&bar[kQFull], qloads & 1, abort_flag, kWaitLimitNs);
+        ++qloads;
         if (!ok) break;
+        mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // the query stage is free again
         tc_fence_after();
-        for (int j = 0; j < pz.npg; ++j) {
-          const int stage = kv_uses % kStages;
-          ok = mbar_wait(&bar[kFull0 + stage], (kv_uses / kStages) & 1, abort_flag, kWaitLimitNs);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t tile = kv_base + stage * kTileBytes;
-          // S = Q . K^T over 576 dims: 9 swizzle blocks x 4 K-steps of 16
-#pragma unroll 4
-          for (int kk = 0; kk < kDqk / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            umma_bf16_ss(tmem + kTmemS, smem_desc_sw128(q_base + off, 16, 1024),
-                         smem_desc_sw128(tile + off, 16, 1024), kIdescQK, kk > 0);
+        ok = issue_qk(first, pages);
+        for (int j = 0; j < pz.npg && ok; ++j) {
+          const int g = pages + j;
+          if (j + 1 < pz.npg) {
+            ok = issue_qk(first + j + 1, g + 1);
+            if (!ok) break;
           }
-          umma_commit(&bar[kSFull]);
-          if (j == pz.npg - 1) umma_commit(&bar[kQEmpty]);
-          ok = mbar_wait(&bar[kPFull], p_uses & 1, abort_flag, kWaitLimitNs);
-          ++p_uses;
+          ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, kWaitLimitNs);
           if (!ok) break;
           tc_fence_after();
+          const int stage = (first + j) % kStages;
+          const uint32_t tile = kv_base + stage * kTileBytes;
           // O += P . V, V = columns 0..511 of the same tile, read MN-major
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
 #pragma unroll
             for (int kk = 0; kk < kPage / 16; ++kk) {
-              umma_bf16_ss(tmem + half * 256, smem_desc_sw128(p_base + kk * 32, 16, 1024),
+              umma_bf16_ss(tmem + kTmemO + half * 256, smem_desc_sw128(p_base + kk * 32, 16, 1024),
                            smem_desc_sw128(tile + half * 4 * kChunkBytes + kk * 2048,
                                            kChunkBytes, 1024),
                            kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(&bar[kEmpty0 + stage]);
-          ++kv_uses;
+          umma_commit(&bar[kPvDone]);
         }
         if (!ok) break;
         umma_commit(&bar[kOFull]);
-        ++pieces_done;
+        pages += pz.npg;
       }
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const bool is_s = lane >= 16;
-    const int r_local = 16 * warp + (lane & 15);
-    const int row = rb * kRowsPerCta + r_local;
-    const bool row_ok = row < p.rows;
-    const int jq = row_ok ? row / p.h_q : 0;
-    const int hq = row_ok ? row % p.h_q : 0;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-    int s_uses = 0, o_uses = 0;
+    // 16-lane TMEM accesses: thread t holds rows t/4 and t/4 + 8 of its quarter's
+    // 16, at columns 2(t%4) + {0,1} + 8g.
+    const uint32_t quarter = static_cast<uint32_t>(32 * warp) << 16;
+    const int ra = 16 * warp + (lane >> 2);
+    const int rbb = ra + 8;
+    const int row_a = rb * kRowsPerCta + ra, row_b = rb * kRowsPerCta + rbb;
+    const bool ok_a = row_a < p.rows, ok_b = row_b < p.rows;
+    const int jq_a = ok_a ? row_a / p.h_q : 0, jq_b = ok_b ? row_b / p.h_q : 0;
+    const int hq_a = ok_a ? row_a % p.h_q : 0, hq_b = ok_b ? row_b % p.h_q : 0;
+    const int c2 = 2 * (lane & 3);
+    const int qr = 16 * warp + lane;  // Q row this thread copies (lanes 0-15)
+    int entries = 0, pages = 0, pieces_done = 0;
     bool ok = true;
     for (int pc = 0; pc < npieces && ok; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       const int L = p.seqlens[pz.seq];
-      int limit = p.causal ? L - p.s_q + jq + 1 : L;
-      limit = limit < 0 ? 0 : (limit > L ? L : limit);
-      if (static_cast<int64_t>(limit) > p.bt_stride * kPage) limit = static_cast<int>(p.bt_stride * kPage);
+      const int cap_tokens = static_cast<int>(p.bt_stride * kPage < L ? p.bt_stride * kPage : L);
+      auto visible = [&](int jq) {
+        int v = p.causal ? L - p.s_q + jq + 1 : L;
+        v = v < 0 ? 0 : v;
+        return v < cap_tokens ? v : cap_tokens;
+      };
+      const int lim_a = visible(jq_a), lim_b = visible(jq_b);
       const int base_split = p.num_splits[pz.seq];
       const int k_pieces = p.num_splits[pz.seq + 1] - base_split;
       const int64_t slot = static_cast<int64_t>(base_split) + pz.split_idx;
-      const int64_t out_row = static_cast<int64_t>(pz.seq) * p.rows + row;
-      float m = -INFINITY, l = 0.f;
+      float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
 
       if (pz.npg > 0) {
+        // ---- query rows: stage -> TMEM lanes 0-15 (lanes 16-31 write the dead O region)
+        const int q_entry = entries;
+        entries += 1 + pz.npg;
+        const int qstage = q_entry % kStages;
+        ok = warp_wait(&bar[kFull0 + qstage], (q_entry / kStages) & 1, abort_flag);
+        if (!ok) break;
+        {
+          const uint8_t* qt = skv + qstage * kTileBytes;
+          for (int c = 0; c < kChunks; ++c) {
+            uint32_t r[32];
+            if (lane < 16) {
+              const uint8_t* rowp = qt + c * kChunkBytes + qr * 128;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((u ^ (qr & 7)) << 4));
+                r[4 * u] = v.x;
+                r[4 * u + 1] = v.y;
+                r[4 * u + 2] = v.z;
+                r[4 * u + 3] = v.w;
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) r[u] = 0u;
+            }
+            tmem_st32(tmem + quarter + kTmemQ + 32 * c, r);
+          }
+          tmem_st_wait();
+        }
+        // Q is in TMEM and the stage has been read: the MMA warp, once all 128
+        // threads have arrived, hands the stage back to the producer.
+        tc_fence_before();
+        mbar_arrive(&bar[kQFull]);
+
         for (int j = 0; j < pz.npg; ++j) {
-          ok = mbar_wait(&bar[kSFull], s_uses & 1, abort_flag, kWaitLimitNs);
-          ++s_uses;
+          const int g = pages + j;
+          ok = warp_wait(&bar[kSFull0 + (g & 1)], (g >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          uint32_t sa[32], sb[32];
-          // 32x32b loads read all 32 lanes of the warp's quarter: lanes 16-31 carry
-          // this page's S row (columns 0..63), lanes 0-15 O values that are unused here.
-          tmem_ld32(tmem + lane_base + 0, sa);
-          tmem_ld32(tmem + lane_base + 32, sb);
-          tmem_ld_wait(sa);
-          tmem_ld_wait(sb);
-          float alpha = 1.f;
-          if (is_s) {
-            const int nvalid_raw = limit - (pz.pg0 + j) * kPage;
-            const int nvalid = nvalid_raw < 0 ? 0 : (nvalid_raw > kPage ? kPage : nvalid_raw);
-            float tmax = -INFINITY;
+          uint32_t s[32];
+          tmem_ld16x64(tmem + quarter + kTmemS + 64 * (g & 1), s);
+          tmem_ld_wait(s);
+          const int tok0 = (pz.pg0 + j) * kPage;
+          const int nv_a = lim_a - tok0, nv_b = lim_b - tok0;
+          float x[32];
+          float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c < nvalid) tmax = fmaxf(tmax, __uint_as_float(sa[c]) * p.scale_log2);
-              if (c + 32 < nvalid) tmax = fmaxf(tmax, __uint_as_float(sb[c]) * p.scale_log2);
-            }
-            float m_new = m;
-            if (tmax > m + kRescaleThreshold) {
-              m_new = tmax;
-              alpha = ex2_approx(m - m_new);  // m = -inf gives 0
-            }
-            float psum = 0.f;
-            uint32_t packed[32];
+          for (int r = 0; r < 32; ++r) {
+            const int tok = c2 + (r & 1) + 8 * (r >> 2);
+            const bool second = (r >> 1) & 1;
+            const bool valid = tok < (second ? nv_b : nv_a);
+            x[r] = valid ? __uint_as_float(s[r]) * p.scale_log2 : -INFINITY;
+            if (second)
+              mx_b = fmaxf(mx_b, x[r]);
+            else
+              mx_a = fmaxf(mx_a, x[r]);
+          }
+          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+          float alpha_a = 1.f, alpha_b = 1.f;
+          if (mx_a > m_a + kRescaleThreshold) {
+            alpha_a = ex2_approx(m_a - mx_a);
+            m_a = mx_a;
+          }
+          if (mx_b > m_b + kRescaleThreshold) {
+            alpha_b = ex2_approx(m_b - mx_b);
+            m_b = mx_b;
+          }
+          float sum_a = 0.f, sum_b = 0.f;
+          uint32_t pw[16];
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float p0 = c < nvalid ? ex2_approx(__uint_as_float(sa[c]) * p.scale_log2 - m_new) : 0.f;
-              const float p1 = c + 1 < nvalid ? ex2_approx(__uint_as_float(sa[c + 1]) * p.scale_log2 - m_new) : 0.f;
-              const float p2 = c + 32 < nvalid ? ex2_approx(__uint_as_float(sb[c]) * p.scale_log2 - m_new) : 0.f;
-              const float p3 = c + 33 < nvalid ? ex2_approx(__uint_as_float(sb[c + 1]) * p.scale_log2 - m_new) : 0.f;
-              psum += (p0 + p1) + (p2 + p3);
-              packed[c >> 1] = pack_bf16x2(p0, p1);
-              packed[16 + (c >> 1)] = pack_bf16x2(p2, p3);
-            }
-            l = l * alpha + psum;
-            m = m_new;
-            // P row r_local: 64 tokens = 8 units of 16 B, 128-byte swizzle
-            uint8_t* prow = sp + r_local * 128;
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float p0 = x[4 * q4] == -INFINITY ? 0.f : ex2_approx(x[4 * q4] - m_a);
+            const float p1 = x[4 * q4 + 1] == -INFINITY ? 0.f : ex2_approx(x[4 * q4 + 1] - m_a);
+            const float p2 = x[4 * q4 + 2] == -INFINITY ? 0.f : ex2_approx(x[4 * q4 + 2] - m_b);
+            const float p3 = x[4 * q4 + 3] == -INFINITY ? 0.f : ex2_approx(x[4 * q4 + 3] - m_b);
+            sum_a += p0 + p1;
+            sum_b += p2 + p3;
+            pw[q4] = pack_bf16x2(p0, p1);
+            pw[8 + q4] = pack_bf16x2(p2, p3);
+          }
+          l_a = l_a * alpha_a + sum_a;
+          l_b = l_b * alpha_b + sum_b;
+          // P and O may be touched only after PV of the previous page is done.
+          if (j > 0) {
+            ok = warp_wait(&bar[kPvDone], (g - 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, alpha_a != 1.f || alpha_b != 1.f)) {
+              for (int cb = 0; cb < kDv; cb += 64) {
+                uint32_t o[32];
+                tmem_ld16x64(tmem + quarter + kTmemO + cb, o);
+                tmem_ld_wait(o);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              uint4 v = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2],
-                                   packed[4 * u + 3]);
-              *reinterpret_cast<uint4*>(prow + ((u ^ (r_local & 7)) << 4)) = v;
+                for (int r = 0; r < 32; ++r)
+                  o[r] = __float_as_uint(__uint_as_float(o[r]) * (((r >> 1) & 1) ? alpha_b : alpha_a));
+                tmem_st16x64(tmem + quarter + kTmemO + cb, o);
+              }
+              tmem_st_wait();
             }
           }
-          const float alpha_o = __shfl_xor_sync(0xffffffffu, alpha, 16);
-          const bool need = (j > 0) && __any_sync(0xffffffffu, (!is_s) && alpha_o != 1.f);
-          if (need) {
-            for (int c0 = 0; c0 < kDv; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_base + c0, o);
-              tmem_ld_wait(o);
-              if (!is_s) {
+          // P rows ra and rbb: token pair (8g + c2, +1) -> 4 bytes in 16-byte unit g (swizzled)
 #pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha_o);
-              }
-              tmem_st32(tmem + lane_base + c0, o);
-            }
-            tmem_st_wait();
+          for (int q4 = 0; q4 < 8; ++q4) {
+            *reinterpret_cast<uint32_t*>(sp + ra * 128 + ((q4 ^ (ra & 7)) << 4) + 2 * c2) = pw[q4];
+            *reinterpret_cast<uint32_t*>(sp + rbb * 128 + ((q4 ^ (rbb & 7)) << 4) + 2 * c2) =
+                pw[8 + q4];
           }
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bar[kPFull]);
         }
         if (!ok) break;
-        ok = mbar_wait(&bar[kOFull], o_uses & 1, abort_flag, kWaitLimitNs);
-        ++o_uses;
+        ok = warp_wait(&bar[kOFull], pieces_done & 1, abort_flag);
+        ++pieces_done;
+        pages += pz.npg;
         if (!ok) break;
         tc_fence_after();
       }
-      // epilogue
-      const float l_o = __shfl_xor_sync(0xffffffffu, l, 16);
-      const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
-      for (int c0 = 0; c0 < kDv; c0 += 32) {
+      // ---- epilogue: the four threads of a row group hold disjoint columns
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      const float inv_a = l_a > 0.f ? 1.f / l_a : 0.f;
+      const float inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
+      const int64_t orow_a = static_cast<int64_t>(pz.seq) * p.rows + row_a;
+      const int64_t orow_b = static_cast<int64_t>(pz.seq) * p.rows + row_b;
+      for (int cb = 0; cb < kDv; cb += 64) {
         uint32_t o[32];
         if (pz.npg > 0) {
-          tmem_ld32(tmem + lane_base + c0, o);
+          tmem_ld16x64(tmem + quarter + kTmemO + cb, o);
           tmem_ld_wait(o);
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
+          for (int r = 0; r < 32; ++r) o[r] = 0u;
         }
-        if (!is_s && row_ok) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int col = cb + 8 * q4 + c2;
+          const float a0 = __uint_as_float(o[4 * q4]) * inv_a;
+          const float a1 = __uint_as_float(o[4 * q4 + 1]) * inv_a;
+          const float b0 = __uint_as_float(o[4 * q4 + 2]) * inv_b;
+          const float b1 = __uint_as_float(o[4 * q4 + 3]) * inv_b;
           if (k_pieces == 1) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + out_row * kDv + c0);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
-              dst[u] = v;
-            }
+            if (ok_a) *reinterpret_cast<uint32_t*>(p.out + orow_a * kDv + col) = pack_bf16x2(a0, a1);
+            if (ok_b) *reinterpret_cast<uint32_t*>(p.out + orow_b * kDv + col) = pack_bf16x2(b0, b1);
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.rows + row) * kDv + c0);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              dst[u] = make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
-                                   __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+            if (ok_a)
+              *reinterpret_cast<float2*>(p.part_o + (slot * p.rows + row_a) * kDv + col) =
+                  make_float2(a0, a1);
+            if (ok_b)
+              *reinterpret_cast<float2*>(p.part_o + (slot * p.rows + row_b) * kDv + col) =
+                  make_float2(b0, b1);
           }
         }
       }
-      if (is_s && row_ok) {
-        const float lse = l > 0.f ? (m + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
-        if (k_pieces == 1)
-          p.lse[(static_cast<int64_t>(pz.seq) * p.h_q + hq) * p.s_q + jq] = lse;
-        else
-          p.part_lse[slot * p.rows + row] = lse;
-      }
-      if (pz.npg > 0) {
-        tc_fence_before();
-        mbar_arrive(&bar[kOFree]);
+      if ((lane & 3) == 0) {
+        const float lse_a = l_a > 0.f ? (m_a + lg2_approx(l_a)) * 0.69314718055994531f : -INFINITY;
+        const float lse_b = l_b > 0.f ? (m_b + lg2_approx(l_b)) * 0.69314718055994531f : -INFINITY;
+        if (k_pieces == 1) {
+          if (ok_a) p.lse[(static_cast<int64_t>(pz.seq) * p.h_q + hq_a) * p.s_q + jq_a] = lse_a;
+          if (ok_b) p.lse[(static_cast<int64_t>(pz.seq) * p.h_q + hq_b) * p.s_q + jq_b] = lse_b;
+        } else {
+          if (ok_a) p.part_lse[slot * p.rows + row_a] = lse_a;
+          if (ok_b) p.part_lse[slot * p.rows + row_b] = lse_b;
+        }
       }
     }
   }
