@@ -29,8 +29,9 @@
 // 0..511).  Softmax, rescale and epilogue use 16-lane TMEM accesses, so they
 // never touch lanes an MMA in flight is writing.
 //
-// Warp roles (192 threads): warps 0-3 softmax/correction/epilogue, warp 4 TMA
-// producer, warp 5 MMA issuer (and TMEM allocator).
+// Warp roles (256 threads): warps 0-3 softmax/correction/epilogue, warp 4 TMA
+// producer, warps 5 and 7 QK^T issuers for even and odd pages (warp 5 also
+// allocates TMEM), warp 6 PV issuer.
 //
 // The method follows "FlashMLA: Revolutionizing Efficient Decoding...",
 // sections 4.2.1-4.2.3 (TMA prefetch of 64-row latent blocks into shared
@@ -44,10 +45,12 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kMmaWarp = 5;    // issues QK^T of even pages; allocates tensor memory
+constexpr int kPvWarp = 6;     // issues PV
+constexpr int kQkOddWarp = 7;  // issues QK^T of odd pages
 constexpr int kChunkBytes = 64 * 128;              // 64 rows x 64 bf16 (one swizzle column block)
 constexpr int kChunks = kDqk / 64;                 // 9
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 73728 = 64 x 576 bf16
@@ -63,6 +66,8 @@ enum Bar {
   kQFull = 2 * kStages,
   kSFull0,
   kSFull1,
+  kSFree0,
+  kSFree1,
   kPFull,
   kPvDone,
   kOFull,
@@ -148,6 +153,8 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar[kQFull], kSoftmaxThreads);
     mbar_init(&bar[kSFull0], 1);
     mbar_init(&bar[kSFull1], 1);
+    mbar_init(&bar[kSFree0], kSoftmaxThreads);
+    mbar_init(&bar[kSFree1], kSoftmaxThreads);
     mbar_init(&bar[kPFull], kSoftmaxThreads);
     mbar_init(&bar[kPvDone], 1);
     mbar_init(&bar[kOFull], 1);
@@ -204,29 +211,17 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_wait(&bar[kFull0 + n % kStages], (n / kStages) & 1, abort_flag, kWaitLimitNs);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kQkOddWarp) {
+    // ------------------------------------------------------------ QK^T issuers
+    // A single thread issues a tcgen05.mma only every ~45 cycles, longer than an
+    // M=64 N=64 MMA takes.  So QK^T of even pages (S buffer 0), QK^T of odd
+    // pages (S buffer 1) and PV come from three warps, and the tensor core runs
+    // their MMAs back to back.  QK^T runs up to two pages ahead of the softmax.
+    const int parity = warp == kMmaWarp ? 0 : 1;
     if (lane == 0) {
       int entries = 0, pages = 0, qloads = 0;
       bool ok = true;
-      const uint32_t kv_base = smem_addr(skv), p_base = smem_addr(sp);
-      auto issue_qk = [&](int entry, int page_index) -> bool {
-        const int stage = entry % kStages;
-        if (!mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint32_t tile = kv_base + stage * kTileBytes;
-        const uint32_t d = tmem + kTmemS + 64 * (page_index & 1);
-        const uint64_t b0 = smem_desc_sw128(tile, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kDqk / 16; ++kk) {
-          // K-step kk: swizzle block kk/4, 32-byte step (kk%4) inside it
-          const uint32_t boff = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-          umma_bf16_ts(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bar[kSFull0 + (page_index & 1)]);
-        return true;
-      };
+      const uint32_t kv_base = smem_addr(skv);
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (pz.npg == 0) continue;
@@ -236,15 +231,47 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = mbar_wait(&bar[kQFull], qloads & 1, abort_flag, kWaitLimitNs);
         ++qloads;
         if (!ok) break;
-        mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // the query stage is free again
+        if (parity == 0) mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // query stage free
         tc_fence_after();
-        ok = issue_qk(first, pages);
         for (int j = 0; j < pz.npg && ok; ++j) {
-          const int g = pages + j;
-          if (j + 1 < pz.npg) {
-            ok = issue_qk(first + j + 1, g + 1);
+          const int g = pages + j, b = g & 1;
+          if (b != parity) continue;
+          if (g >= 2) {  // the softmax has read S of page g - 2 from buffer b
+            ok = mbar_wait(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag, kWaitLimitNs);
             if (!ok) break;
           }
+          const int entry = first + j, stage = entry % kStages;
+          ok = mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t b0 = smem_desc_sw128(kv_base + stage * kTileBytes, 16, 1024);
+          const uint32_t d = tmem + kTmemS + 64 * b;
+#pragma unroll
+          for (int kk = 0; kk < kDqk / 16; ++kk) {
+            // K-step kk: swizzle block kk/4, 32-byte step (kk%4) inside it
+            const uint32_t boff = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+            umma_bf16_ts(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar[kSFull0 + b]);
+        }
+        pages += pz.npg;
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      int entries = 0, pages = 0;
+      bool ok = true;
+      const uint32_t kv_base = smem_addr(skv), p_base = smem_addr(sp);
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (pz.npg == 0) continue;
+        const int first = entries + 1;
+        entries += 1 + pz.npg;
+        for (int j = 0; j < pz.npg; ++j) {
+          const int g = pages + j;
+          // P of page g is in shared memory (and QK^T of page g, which read the
+          // same stage, has completed: the softmax saw its S)
           ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, kWaitLimitNs);
           if (!ok) break;
           tc_fence_after();
@@ -265,6 +292,8 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           umma_commit(&bar[kPvDone]);
         }
         if (!ok) break;
+        // every MMA of the piece is complete once this fires: the last PV
+        // follows (through the softmax) the last QK^T
         umma_commit(&bar[kOFull]);
         pages += pz.npg;
       }
@@ -341,6 +370,8 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           uint32_t s[32];
           tmem_ld16x64(tmem + quarter + kTmemS + 64 * (g & 1), s);
           tmem_ld_wait(s);
+          tc_fence_before();
+          mbar_arrive(&bar[kSFree0 + (g & 1)]);
           const int tok0 = (pz.pg0 + j) * kPage;
           const int nv_a = lim_a - tok0, nv_b = lim_b - tok0;
           float x[32];
