@@ -64,11 +64,19 @@ def assert_close_lse(got, ref, where=""):
                              f"(neg-inf mismatch: {int((np.isneginf(got) != np.isneginf(ref)).sum())})")
 
 
+def workers_used(res, dev, inp, num_workers):
+    W = int(res["tile_md"].shape[0])
+    if num_workers is not None:
+        assert W == num_workers
+    else:
+        assert 1 <= W <= expected_workers(dev, inp.s_q, inp.h_q)
+    return W
+
+
 def full_parity(inp, dev, num_workers=None):
     res = run_cuda(inp, dev, num_workers)
     assert res["status"] == 0, f"device status {res['status']}"
-    W = num_workers if num_workers is not None else expected_workers(dev, inp.s_q, inp.h_q)
-    assert res["tile_md"].shape[0] == W
+    W = workers_used(res, dev, inp, num_workers)
     check_metadata(inp, res, W)
     ref_out, ref_lse = oracle.decode(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens,
                                      inp.scale, inp.causal)
@@ -82,7 +90,7 @@ def sampled_parity(inp, dev, n_rows=64, seed=0, extra_rows=()):
     a random sample of output rows one by one."""
     res = run_cuda(inp, dev)
     assert res["status"] == 0, f"device status {res['status']}"
-    W = expected_workers(dev, inp.s_q, inp.h_q)
+    W = workers_used(res, dev, inp, None)
     check_metadata(inp, res, W)
     g = np.random.default_rng(seed)
     b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
