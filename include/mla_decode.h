@@ -64,9 +64,13 @@ typedef enum {
 /*
  * mla_metadata_shape -- sizes for the split-KV metadata.
  *
- * num_workers: how many workers the decode grid uses on the current device:
- *   max(1, SMs / ceil(s_q * h_q / 64)).  One worker is one CTA per 64-row block
- *   of the query rows.  md_stride: MLA_MD_STRIDE.
+ * num_workers: how many workers the decode grid uses on the current device.
+ *   With s_q * h_q <= 64 query rows per sequence, one worker is one CTA and
+ *   num_workers = SMs.  With more rows, one worker is one pair of CTAs (a
+ *   cluster of 2) per 128-row block: num_workers = min(SMs / (2 B),
+ *   C / B) with B = ceil(s_q * h_q / 128) and C the number of pairs of the
+ *   decode kernel the device holds at once, so that every pair of the grid
+ *   runs in the first wave.  At least 1.  md_stride: MLA_MD_STRIDE.
  * Returns MLA_OK, MLA_ERR_INVALID_ARG (batch, h_q or s_q < 1, null outputs), or
  * MLA_ERR_CUDA (no current device).
  */

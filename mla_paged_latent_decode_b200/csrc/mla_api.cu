@@ -46,7 +46,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // A [rows, 576] bf16 row-major matrix read in (box_rows x 64) boxes with 128-byte swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows = 64) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(rows)};
@@ -61,9 +61,24 @@ bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t bo
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int row_blocks(int s_q, int h_q) {
+// Query rows up to 64 per sequence run on single CTAs (one 64-row block); more
+// rows run on CTA pairs, one pair per 128-row block.
+bool uses_pairs(int s_q, int h_q) { return static_cast<int64_t>(s_q) * h_q > mla::kRowsPerCta; }
+
+int workers_for(int sms, int s_q, int h_q, int* out) {
   const int rows = s_q * h_q;
-  return (rows + mla::kRowsPerCta - 1) / mla::kRowsPerCta;
+  if (!uses_pairs(s_q, h_q)) {
+    *out = sms > 1 ? sms : 1;
+    return MLA_OK;
+  }
+  const int blocks128 = (rows + 127) / 128;
+  int clusters = 0;
+  if (mla::pair_kernel_max_clusters(&clusters) != cudaSuccess) return MLA_ERR_CUDA;
+  int w = sms / (2 * blocks128);
+  const int w_fit = clusters / blocks128;  // every pair of the grid resident at once
+  if (w_fit < w) w = w_fit;
+  *out = w > 1 ? w : 1;
+  return MLA_OK;
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -88,7 +103,7 @@ const char* mla_error_string(int status) {
 }
 
 const char* mla_version(void) {
-  return "mla_paged_latent_decode_b200 sm_100a (tcgen05 M=64 decode, Q in TMEM, 3-stage TMA)";
+  return "mla_paged_latent_decode_b200 sm_100a (tcgen05 pair decode for >64 query rows, M=64 decode otherwise)";
 }
 
 int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_stride) {
@@ -98,8 +113,8 @@ int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_st
   int sms = 0;
   int rc = current_sm_count(&sms);
   if (rc != MLA_OK) return rc;
-  const int rb = row_blocks(s_q, h_q);
-  *num_workers = sms / rb > 1 ? sms / rb : 1;
+  rc = workers_for(sms, s_q, h_q, num_workers);
+  if (rc != MLA_OK) return rc;
   *md_stride = MLA_MD_STRIDE;
   return MLA_OK;
 }
@@ -150,8 +165,8 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
 
   const int rows = s_q * h_q;
   CUtensorMap tm_q, tm_kv;
-  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows, 64)) return MLA_ERR_CUDA;
-  if (!make_row_map(&tm_kv, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage, 64))
+  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
+  if (!make_row_map(&tm_kv, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage))
     return MLA_ERR_CUDA;
 
   const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
@@ -179,7 +194,15 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (mla::launch_decode(tm_q, tm_kv, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (uses_pairs(s_q, h_q)) {
+    CUtensorMap tm_k32;
+    if (!make_row_map(&tm_k32, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage, 32))
+      return MLA_ERR_CUDA;
+    if (mla::launch_decode_pair(tm_q, tm_k32, tm_kv, p, num_workers, st) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  } else {
+    if (mla::launch_decode(tm_q, tm_kv, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
+  }
 
   mla::CombineParams c{};
   c.num_splits = num_splits;

@@ -1,0 +1,682 @@
+// mla_decode_pair_sm100.cu -- MLA decode on CTA pairs (clusters of 2), sm_100a.
+//
+// Used when a sequence has more than 64 query rows (s_q * h_q > 64).  A pair
+// of CTAs owns a 128-row block of the query rows of one worker's run of
+// (sequence, page) items; CTA r of the pair holds rows 64r..64r+63.  Every MMA
+// is a pair MMA (tcgen05 .cta_group::2, M = 128 rows split over the two SMs),
+// which runs at the full rate of the tensor cores, where the single-CTA kernel
+// for narrow rows (mla_decode_sm100.cu) issues half-rate M=64 MMAs.
+//
+// Per page (64 tokens x 576 bf16):
+//   S  = Q . K^T   N = 64 tokens: CTA r supplies tokens 32r..32r+31 of the page
+//                  (all 576 dims) as its half of B; each CTA receives S for its
+//                  64 rows and all 64 tokens.  Dims 0..383 of Q are read from
+//                  tensor memory, dims 384..575 from shared memory.
+//   O += P . V     N = 256 dv per MMA, two MMAs: CTA r supplies, for all 64
+//                  tokens, dv 256h+128r .. 256h+128r+127 of MMA h as its half of B.
+// So each CTA loads its 32 token rows in full (K part, 36 KB) and its 256
+// columns of dv for all 64 tokens (V part, 32 KB); the two CTAs together read
+// each page from HBM once.  Both parts are TMA boxes through the block table,
+// with 128-byte swizzle; their completion is counted on the leader's barriers.
+//
+// Tensor memory per CTA (512 columns, all 128 lanes):
+//   O   columns   0..255  64 rows x 512 fp32: lane L holds row L % 64, dv half
+//                         L / 64 of each 256-wide MMA
+//   S   columns 256..319  two buffers of 32 columns: lane L, row L % 64,
+//                         tokens 32 (L / 64) + c
+//   Q   columns 320..511  dims 0..383 of the 64 rows, two bf16 per column, each
+//                         row held in lanes L and L + 64
+// The rest of Q (dims 384..575, 24 KB) stays in shared memory, which leaves room
+// for three K-part slots, two V-part slots and two P buffers.
+//
+// The K-part ring also stages the query rows: per piece, two ring entries carry
+// dims 0..255 and 256..383 of this CTA's 64 rows (plain TMA, counted on this
+// CTA's own barrier); the softmax warps copy them into tensor memory, and the
+// leader's QK^T warp releases both slots once the copies of both CTAs are done.
+//
+// Warp roles (288 threads per CTA):
+//   warps 0-3  softmax / correction / epilogue (both CTAs); thread L owns half
+//              of row L % 64; the two halves of a row exchange maxima and sums
+//              through shared memory.
+//   warp 4     TMA: query rows and K parts (both CTAs).
+//   warp 8     TMA: V parts (both CTAs).
+//   warps 5, 7 QK^T of even / odd pages (leader CTA only); warp 5 also
+//              allocates the pair's tensor memory in each CTA.
+//   warp 6     PV (leader CTA only).
+// P is double-buffered, so the softmax of page g overlaps PV of page g - 1; the
+// softmax waits for that PV only when it has to rescale O.
+//
+// The method is that of the single-CTA kernel ("FlashMLA: Revolutionizing
+// Efficient Decoding...", sections 4.2.1-4.2.3: TMA prefetch of 64-row latent
+// blocks, tensor cores for QK^T and PV, softmax fused in the kernel), mapped
+// onto the pair tensor-core instructions of sm_100a.
+#include "mla_kernels.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int kThreads = 288;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kTmaKWarp = 4;
+constexpr int kQkEvenWarp = 5;
+constexpr int kPvWarp = 6;
+constexpr int kQkOddWarp = 7;
+constexpr int kTmaVWarp = 8;
+
+constexpr int kChunk = 64 * 128;          // 64 rows x 64 bf16 (one 128-byte swizzle column block)
+constexpr int kHalfChunk = 32 * 128;      // 32 rows x 64 bf16
+constexpr int kChunks = kDqk / 64;        // 9
+constexpr int kQTmemChunks = 6;           // dims 0..383 of Q live in tensor memory
+constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // dims 384..575 stay in shared memory
+constexpr int kQStageA = 4;               // first staging entry: chunks 0..3
+constexpr int kQ2Bytes = kQSmemChunks * kChunk;        // 24576
+constexpr int kKBytes = kChunks * kHalfChunk;          // 36864: 32 tokens x 576
+constexpr int kVBytes = 4 * kChunk;                    // 32768: 64 tokens x 256 dv
+constexpr int kPBytes = kChunk;                        // 64 rows x 64 tokens
+constexpr int kKSlots = 3;
+constexpr int kVSlots = 2;
+constexpr int kQKSteps = kDqk / 16;                    // 36
+constexpr int kQTmemKSteps = kQTmemChunks * 4;         // 24
+static_assert(kQStageA * kChunk <= kKBytes && (kQTmemChunks - kQStageA) * kChunk <= kKBytes,
+              "query staging entries fit a K-part slot");
+
+constexpr int kOffQ2 = 0;
+constexpr int kOffK = kOffQ2 + kQ2Bytes;
+constexpr int kOffV = kOffK + kKSlots * kKBytes;
+constexpr int kOffP = kOffV + kVSlots * kVBytes;
+constexpr int kOffX = kOffP + 2 * kPBytes;       // row-half exchange: [2 pages][2 halves][64] f32
+constexpr int kOffL = kOffX + 2 * 2 * 64 * 4;    // epilogue sum exchange: [2 pieces][2 halves][64] f32
+constexpr int kOffBar = kOffL + 2 * 2 * 64 * 4;
+static_assert(kOffK % 1024 == 0 && kKBytes % 1024 == 0 && kOffV % 1024 == 0 &&
+                  kOffP % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
+enum Bar {
+  kKFull0 = 0,                                    // leader: K parts of both CTAs
+  kVFull0 = kKFull0 + kKSlots,                    // leader: V parts of both CTAs
+  kQFull = kVFull0 + kVSlots,                     // leader: Q dims 384..575 of both CTAs
+  kKEmpty0,                                       // both: pair commits (multicast)
+  kVEmpty0 = kKEmpty0 + kKSlots,
+  kQEmpty = kVEmpty0 + kVSlots,
+  kSFull0, kSFull1, kPvDone0, kPvDone1, kOFull,   // both: pair commits (multicast)
+  kSFree0, kSFree1, kPFull0, kPFull1, kQReady,    // leader: softmax warps of both CTAs
+  kQStage,                                        // local: this CTA's query staging copies
+  kXBar, kLBar,                                   // local: softmax exchanges
+  kNumBars
+};
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemUsed = kOffMisc + 16;
+constexpr int kSmemBytes = kSmemUsed + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 0;       // 256 columns
+constexpr uint32_t kTmemS = 256;     // S buffer b at 256 + 32 b
+constexpr uint32_t kTmemQ = 320;     // 192 columns
+static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "tensor memory budget");
+constexpr float kRescaleThreshold = 8.0f;
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
+constexpr uint32_t kSoftmaxArrivals = 2 * kSoftmaxWarps;   // one per softmax warp, both CTAs
+
+struct Piece {
+  int seq, pg0, npg, split_idx;
+};
+
+__device__ __forceinline__ Piece piece_of(const int32_t* md, int pc, const int32_t* seqlens,
+                                          int64_t bt_stride) {
+  const int npieces = md[5];
+  Piece p;
+  p.seq = md[0] + pc;
+  const int L = seqlens[p.seq];
+  int npages = L > 0 ? (L + kPage - 1) / kPage : 0;
+  if (npages > bt_stride) npages = static_cast<int>(bt_stride);
+  const int it0 = pc == 0 ? md[1] : 0;
+  const int it1 = pc == npieces - 1 ? md[3] : (npages > 0 ? npages : 1);
+  const int pg1 = it1 < npages ? it1 : npages;
+  p.pg0 = it0;
+  p.npg = pg1 > it0 ? pg1 - it0 : 0;
+  p.split_idx = pc == 0 ? md[4] : 0;
+  return p;
+}
+
+__device__ __forceinline__ void report(int32_t* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort, kWaitLimitNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// One arrival per warp on a barrier of the pair leader (CTA 0).
+__device__ __forceinline__ void warp_arrive_leader(uint64_t* bar, uint32_t rank, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    if (rank == 0)
+      mbar_arrive(bar);
+    else
+      mbar_arrive_remote(bar, 0);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k32,
+                       const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sq2 = smem + kOffQ2;
+  uint8_t* sk = smem + kOffK;
+  uint8_t* sv = smem + kOffV;
+  uint8_t* sp = smem + kOffP;
+  float* sx = reinterpret_cast<float*>(smem + kOffX);
+  float* sl = reinterpret_cast<float*>(smem + kOffL);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int worker = blockIdx.x >> 1, rb2 = blockIdx.y;
+  const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
+  const int npieces = md[5];
+  if (npieces == 0) return;  // idle worker: both CTAs of the pair leave together
+  if (md[0] < 0 || npieces < 0 || md[0] + npieces > p.batch) {
+    if (threadIdx.x == 0 && rank == 0) report(p.status, MLA_ERR_DEVICE_CHECK);
+    return;
+  }
+  const int row0 = rb2 * 128 + 64 * static_cast<int>(rank);  // first query row of this CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&bar[kKFull0 + s], 1);
+      mbar_init(&bar[kKEmpty0 + s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(&bar[kVFull0 + s], 1);
+      mbar_init(&bar[kVEmpty0 + s], 1);
+    }
+    mbar_init(&bar[kQFull], 1);
+    mbar_init(&bar[kQEmpty], 2);  // one commit from each QK^T warp
+    mbar_init(&bar[kSFull0], 1);
+    mbar_init(&bar[kSFull1], 1);
+    mbar_init(&bar[kPvDone0], 1);
+    mbar_init(&bar[kPvDone1], 1);
+    mbar_init(&bar[kOFull], 1);
+    mbar_init(&bar[kSFree0], kSoftmaxArrivals);
+    mbar_init(&bar[kSFree1], kSoftmaxArrivals);
+    mbar_init(&bar[kPFull0], kSoftmaxArrivals);
+    mbar_init(&bar[kPFull1], kSoftmaxArrivals);
+    mbar_init(&bar[kQReady], kSoftmaxArrivals);
+    mbar_init(&bar[kQStage], 1);
+    mbar_init(&bar[kXBar], 32 * kSoftmaxWarps);
+    mbar_init(&bar[kLBar], 32 * kSoftmaxWarps);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kQkEvenWarp) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers and tensor memory of both CTAs exist before either uses them
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Every role walks the same sequence of K-ring entries: per piece with pages,
+  // two query-staging entries, then one entry per page.
+  if (warp == kTmaKWarp) {
+    // ------------------------------------------------------------ query rows + K parts
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k32);
+      int entries = 0, qloads = 0;
+      bool ok = true;
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (rank == 0 && p.seqlens[pz.seq] > p.bt_stride * kPage)
+          report(p.status, MLA_ERR_DEVICE_CHECK);
+        if (pz.npg == 0) continue;
+        const int qrow = pz.seq * p.rows + row0;
+        // dims 384..575 of the query rows: shared memory, counted on the leader
+        if (qloads > 0) {
+          ok = mbar_wait_cluster(&bar[kQEmpty], (qloads - 1) & 1, abort_flag, kWaitLimitNs);
+          if (!ok) break;
+        }
+        if (rank == 0) mbar_arrive_expect_tx(&bar[kQFull], 2 * kQ2Bytes);
+        for (int c = 0; c < kQSmemChunks; ++c)
+          tma_load_2d_pair(sq2 + c * kChunk, &tm_q, (kQTmemChunks + c) * 64, qrow, &bar[kQFull]);
+        ++qloads;
+        // dims 0..383: two staging entries of the K ring, counted on this CTA's barrier
+        for (int e = 0; e < 2; ++e) {
+          const int slot = entries % kKSlots, use = entries / kKSlots;
+          if (use > 0) {
+            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
+                                   kWaitLimitNs);
+            if (!ok) break;
+          }
+          if (e == 0) mbar_arrive_expect_tx(&bar[kQStage], kQTmemChunks * kChunk);
+          uint8_t* dst = sk + slot * kKBytes;
+          const int c0 = e == 0 ? 0 : kQStageA, c1 = e == 0 ? kQStageA : kQTmemChunks;
+          for (int c = c0; c < c1; ++c)
+            tma_load_2d(dst + (c - c0) * kChunk, &tm_q, c * 64, qrow, &bar[kQStage]);
+          // the leader's full barrier of the slot completes one phase per entry
+          if (rank == 0) mbar_arrive(&bar[kKFull0 + slot]);
+          ++entries;
+        }
+        if (!ok) break;
+        const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+        for (int j = 0; j < pz.npg; ++j, ++entries) {
+          const int slot = entries % kKSlots, use = entries / kKSlots;
+          if (use > 0) {
+            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
+                                   kWaitLimitNs);
+            if (!ok) break;
+          }
+          const int page = __ldg(bt + pz.pg0 + j);
+          if (rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
+          uint8_t* dst = sk + slot * kKBytes;
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_2d_pair(dst + c * kHalfChunk, &tm_k32, c * 64,
+                             page * kPage + 32 * static_cast<int>(rank), &bar[kKFull0 + slot]);
+        }
+      }
+    }
+  } else if (warp == kTmaVWarp) {
+    // ------------------------------------------------------------ V parts
+    if (lane == 0) {
+      prefetch_tensormap(&tm_kv);
+      int pages = 0;
+      bool ok = true;
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (pz.npg == 0) continue;
+        const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+        for (int j = 0; j < pz.npg; ++j, ++pages) {
+          const int slot = pages % kVSlots, use = pages / kVSlots;
+          if (use > 0) {
+            ok = mbar_wait_cluster(&bar[kVEmpty0 + slot], (use - 1) & 1, abort_flag,
+                                   kWaitLimitNs);
+            if (!ok) break;
+          }
+          const int page = __ldg(bt + pz.pg0 + j);
+          if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kVBytes);
+          uint8_t* dst = sv + slot * kVBytes;
+          // sub-chunk 2h + e holds dv block 4h + 2 rank + e (64 dv each)
+          for (int h = 0; h < 2; ++h)
+            for (int e = 0; e < 2; ++e)
+              tma_load_2d_pair(dst + (2 * h + e) * kChunk, &tm_kv,
+                               64 * (4 * h + 2 * static_cast<int>(rank) + e), page * kPage,
+                               &bar[kVFull0 + slot]);
+        }
+      }
+    }
+  } else if (warp == kQkEvenWarp || warp == kQkOddWarp) {
+    // ------------------------------------------------------------ QK^T issuers (leader)
+    // One thread issues a tcgen05.mma at most every ~45 cycles; even and odd
+    // pages (one S buffer each) come from two warps so the tensor core stays fed.
+    if (rank == 0 && lane == 0) {
+      const int parity = warp == kQkEvenWarp ? 0 : 1;
+      int entries = 0, pages = 0, qloads = 0;
+      bool ok = true;
+      const uint32_t q2_base = smem_addr(sq2), k_base = smem_addr(sk);
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (pz.npg == 0) continue;
+        const int stage_a = entries % kKSlots, stage_b = (entries + 1) % kKSlots;
+        entries += 2;
+        ok = mbar_wait_cluster(&bar[kQFull], qloads & 1, abort_flag, kWaitLimitNs) &&
+             mbar_wait_cluster(&bar[kQReady], qloads & 1, abort_flag, kWaitLimitNs);
+        ++qloads;
+        if (!ok) break;
+        tc_fence_after();
+        if (parity == 0) {  // both CTAs hold Q in tensor memory: the staging slots are free
+          umma_commit_pair(&bar[kKEmpty0 + stage_a]);
+          umma_commit_pair(&bar[kKEmpty0 + stage_b]);
+        }
+        for (int j = 0; j < pz.npg && ok; ++j) {
+          const int g = pages + j, b = g & 1, entry = entries + j;
+          if (b != parity) continue;
+          if (g >= 2) {  // both CTAs' softmax have read S of page g - 2 from buffer b
+            ok = mbar_wait_cluster(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag,
+                                   kWaitLimitNs);
+            if (!ok) break;
+          }
+          const int slot = entry % kKSlots;
+          ok = mbar_wait_cluster(&bar[kKFull0 + slot], (entry / kKSlots) & 1, abort_flag,
+                                 kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t b0 = smem_desc_sw128(k_base + slot * kKBytes, 16, 1024);
+          const uint64_t a2 = smem_desc_sw128(q2_base, 16, 1024);
+          const uint32_t d = tmem + kTmemS + 32 * b;
+#pragma unroll
+          for (int kk = 0; kk < kQKSteps; ++kk) {
+            // K-step kk: swizzle block kk/4, 32-byte step kk%4 inside it
+            const uint32_t boff = ((kk >> 2) * kHalfChunk + (kk & 3) * 32) >> 4;
+            if (kk < kQTmemKSteps) {
+              umma_bf16_ts_pair(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
+            } else {
+              const int k2 = kk - kQTmemKSteps;
+              const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
+              umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
+            }
+          }
+          umma_commit_pair(&bar[kSFull0 + b]);
+          umma_commit_pair(&bar[kKEmpty0 + slot]);
+        }
+        if (!ok) break;
+        umma_commit_pair(&bar[kQEmpty]);  // this warp's reads of Q for the piece are done
+        entries += pz.npg;
+        pages += pz.npg;
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV issuer (leader)
+    if (rank == 0 && lane == 0) {
+      int pages = 0;
+      bool ok = true;
+      const uint32_t v_base = smem_addr(sv), p_base = smem_addr(sp);
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (pz.npg == 0) continue;
+        for (int j = 0; j < pz.npg; ++j) {
+          const int g = pages + j, slot = g % kVSlots, pb = g & 1;
+          ok = mbar_wait_cluster(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, kWaitLimitNs);
+          if (!ok) break;
+          ok = mbar_wait_cluster(&bar[kVFull0 + slot], (g / kVSlots) & 1, abort_flag,
+                                 kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vt = v_base + slot * kVBytes;
+          const uint32_t pt = p_base + pb * kPBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int kk = 0; kk < kPage / 16; ++kk) {
+              umma_bf16_ss_pair(tmem + kTmemO + 128 * h, smem_desc_sw128(pt + kk * 32, 16, 1024),
+                                smem_desc_sw128(vt + 2 * h * kChunk + kk * 2048, kChunk, 1024),
+                                kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit_pair(&bar[kVEmpty0 + slot]);
+          umma_commit_pair(&bar[kPvDone0 + pb]);
+        }
+        if (!ok) break;
+        umma_commit_pair(&bar[kOFull]);
+        pages += pz.npg;
+      }
+    }
+  } else if (warp < kSoftmaxWarps) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int L = 32 * warp + lane;       // TMEM lane
+    const int r = L & 63;                 // row within this CTA's 64
+    const int th = L >> 6;                // which half of the 64 tokens / of each dv 256-block
+    const int row = row0 + r;             // row within the sequence's query rows
+    const bool row_ok = row < p.rows;
+    const int jq = row_ok ? row / p.h_q : 0, hq = row_ok ? row % p.h_q : 0;
+    const uint32_t quarter = static_cast<uint32_t>(32 * warp) << 16;
+    int entries = 0, pages = 0, pieces_done = 0, qcopies = 0;
+    bool ok = true;
+    for (int pc = 0; pc < npieces && ok; ++pc) {
+      const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+      const int Lseq = p.seqlens[pz.seq];
+      const int cap_tokens =
+          static_cast<int>(p.bt_stride * kPage < Lseq ? p.bt_stride * kPage : Lseq);
+      int lim = p.causal ? Lseq - p.s_q + jq + 1 : Lseq;
+      lim = lim < 0 ? 0 : (lim < cap_tokens ? lim : cap_tokens);
+      const int base_split = p.num_splits[pz.seq];
+      const int k_pieces = p.num_splits[pz.seq + 1] - base_split;
+      const int64_t slot = static_cast<int64_t>(base_split) + pz.split_idx;
+      float m = -INFINITY, l = 0.f;
+
+      if (pz.npg > 0) {
+        // ---- query dims 0..383: staging slots -> tensor memory (row r in lanes r, r + 64).
+        // Both QK^T warps have finished the previous piece (their Q-empty commit),
+        // so no MMA still reads the old rows and neither warp can miss a phase
+        // of the Q-ready barrier.
+        {
+          const uint8_t* qa = sk + (entries % kKSlots) * kKBytes;
+          const uint8_t* qb = sk + ((entries + 1) % kKSlots) * kKBytes;
+          entries += 2;
+          if (qcopies > 0) {
+            ok = warp_wait_cluster(&bar[kQEmpty], (qcopies - 1) & 1, abort_flag);
+            if (!ok) break;
+          }
+          ok = warp_wait_cluster(&bar[kQStage], qcopies & 1, abort_flag);
+          ++qcopies;
+          if (!ok) break;
+          for (int c = 0; c < kQTmemChunks; ++c) {
+            const uint8_t* rowp =
+                (c < kQStageA ? qa + c * kChunk : qb + (c - kQStageA) * kChunk) + r * 128;
+            uint32_t q[32];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((u ^ (r & 7)) << 4));
+              q[4 * u] = v.x;
+              q[4 * u + 1] = v.y;
+              q[4 * u + 2] = v.z;
+              q[4 * u + 3] = v.w;
+            }
+            tmem_st32(tmem + quarter + kTmemQ + 32 * c, q);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          warp_arrive_leader(&bar[kQReady], rank, lane);
+        }
+        for (int j = 0; j < pz.npg; ++j) {
+          const int g = pages + j, pb = g & 1;
+          ok = warp_wait_cluster(&bar[kSFull0 + pb], (g >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t s[32];
+          tmem_ld32(tmem + quarter + kTmemS + 32 * pb, s);
+          tmem_ld_wait(s);
+          tc_fence_before();
+          warp_arrive_leader(&bar[kSFree0 + pb], rank, lane);
+          const int nv = lim - (pz.pg0 + j) * kPage - 32 * th;
+          float x[32];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[c] = c < nv ? __uint_as_float(s[c]) * p.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, x[c]);
+          }
+          // the other half of the row is in lane L ^ 64
+          float* xb = sx + pb * 128;
+          xb[th * 64 + r] = mx;
+          mbar_arrive(&bar[kXBar]);
+          ok = warp_wait_cluster(&bar[kXBar], g & 1, abort_flag);
+          if (!ok) break;
+          mx = fmaxf(mx, xb[(th ^ 1) * 64 + r]);
+          float alpha = 1.f;
+          if (mx > m + kRescaleThreshold) {
+            alpha = ex2_approx(m - mx);
+            m = mx;
+          }
+          float sum = 0.f;
+          uint32_t pw[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = x[c] == -INFINITY ? 0.f : ex2_approx(x[c] - m);
+            const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_approx(x[c + 1] - m);
+            sum += p0 + p1;
+            pw[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          l = l * alpha + sum;
+          // O is rescaled only once PV of the previous page is done; the first
+          // PV of a piece overwrites O, so its page needs no rescale.
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            ok = warp_wait_cluster(&bar[kPvDone0 + ((g - 1) & 1)], ((g - 1) >> 1) & 1,
+                                   abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            for (int cb = 0; cb < 256; cb += 32) {
+              uint32_t o[32];
+              tmem_ld32(tmem + quarter + kTmemO + cb, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(tmem + quarter + kTmemO + cb, o);
+            }
+            tmem_st_wait();
+          }
+          // P buffer pb was last read by PV of page g - 2
+          if (g >= 2) {
+            ok = warp_wait_cluster(&bar[kPvDone0 + pb], ((g >> 1) - 1) & 1, abort_flag);
+            if (!ok) break;
+          }
+          // P row r, tokens 32 th .. 32 th + 31: 16-byte units 4 th .. 4 th + 3 (swizzled)
+          uint8_t* prow = sp + pb * kPBytes + r * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int u = 4 * th + i;
+            *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
+                make_uint4(pw[4 * i], pw[4 * i + 1], pw[4 * i + 2], pw[4 * i + 3]);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          warp_arrive_leader(&bar[kPFull0 + pb], rank, lane);
+        }
+        if (!ok) break;
+        ok = warp_wait_cluster(&bar[kOFull], pieces_done & 1, abort_flag);
+        ++pieces_done;
+        entries += pz.npg;
+        pages += pz.npg;
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // ---- epilogue: sums of the two row halves, then O / l
+      float* lb = sl + (pc & 1) * 128;
+      lb[th * 64 + r] = l;
+      mbar_arrive(&bar[kLBar]);
+      ok = warp_wait_cluster(&bar[kLBar], pc & 1, abort_flag);
+      if (!ok) break;
+      const float lt = l + lb[(th ^ 1) * 64 + r];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const int64_t orow = static_cast<int64_t>(pz.seq) * p.rows + row;
+      for (int h = 0; h < 2; ++h) {
+        const int dv0 = 256 * h + 128 * th;
+        for (int cb = 0; cb < 128; cb += 32) {
+          uint32_t o[32];
+          if (pz.npg > 0) {
+            tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb, o);
+            tmem_ld_wait(o);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          }
+          if (!row_ok) continue;
+          if (k_pieces == 1) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + dv0 + cb);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[8 * u]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+              dst[u] = v;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.rows + row) * kDv + dv0 + cb);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              dst[u] = make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                                   __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+          }
+        }
+      }
+      if (row_ok && th == 0) {
+        const float lse = lt > 0.f ? (m + lg2_approx(lt)) * 0.69314718055994531f : -INFINITY;
+        if (k_pieces == 1)
+          p.lse[(static_cast<int64_t>(pz.seq) * p.h_q + hq) * p.s_q + jq] = lse;
+        else
+          p.part_lse[slot * p.rows + row] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no pair MMA still writes either CTA's tensor memory
+  if (*abort_flag && threadIdx.x == 0) report(p.status, MLA_ERR_DEVICE_TIMEOUT);
+  if (warp == kQkEvenWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k32,
+                               const CUtensorMap& tm_kv, const DecodeParams& p, int num_workers,
+                               cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int blocks128 = (p.rows + 127) / 128;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * num_workers, blocks128, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_k32, tm_kv, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Pairs (clusters of 2) of this kernel that fit on the device at once.
+cudaError_t pair_kernel_max_clusters(int* clusters) {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (cached[dev] > 0) {
+    *clusters = cached[dev];
+    return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  if (n < 1) n = 1;
+  cached[dev] = n;
+  *clusters = n;
+  return cudaSuccess;
+}
+
+}  // namespace mla

@@ -71,7 +71,12 @@ def split_plan(seqlens, num_workers: int):
     return md, num_splits
 
 
-def num_workers_for(num_sms: int, s_q: int, h_q: int, rows_per_cta: int = 64) -> int:
-    """Workers the decode grid uses: one CTA per SM, shared among the 64-row blocks."""
-    row_blocks = -(-(s_q * h_q) // rows_per_cta)
-    return max(1, num_sms // row_blocks)
+def num_workers_for(num_sms: int, s_q: int, h_q: int) -> int:
+    """Upper bound on the workers the decode grid uses: one CTA per SM for up to
+    64 query rows, else one pair of CTAs per 128-row block (the library may use
+    fewer pairs, as many as the device holds at once)."""
+    rows = s_q * h_q
+    if rows <= 64:
+        return max(1, num_sms)
+    blocks = -(-rows // 128)
+    return max(1, num_sms // (2 * blocks))

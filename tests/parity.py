@@ -69,7 +69,7 @@ def workers_used(res, dev, inp, num_workers):
     if num_workers is not None:
         assert W == num_workers
     else:
-        assert W == expected_workers(dev, inp.s_q, inp.h_q)
+        assert 1 <= W <= expected_workers(dev, inp.s_q, inp.h_q)
     return W
 
 
