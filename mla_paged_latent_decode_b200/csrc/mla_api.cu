@@ -59,6 +59,23 @@ bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t bo
   return r == CUDA_SUCCESS;
 }
 
+// The fp32 partial outputs [slots, rows, 512] written in 32 x 32 boxes with
+// 128-byte swizzle; the row extent clips boxes that run past a sequence's rows.
+bool make_partial_map(CUtensorMap* map, float* base, uint64_t rows, uint64_t slots) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDv), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(slots)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDv) * 4,
+                           static_cast<cuuint64_t>(mla::kDv) * 4 * rows};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Query rows up to 64 per sequence run on single CTAs (one 64-row block); more
@@ -198,7 +215,9 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
     CUtensorMap tm_k32;
     if (!make_row_map(&tm_k32, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage, 32))
       return MLA_ERR_CUDA;
-    if (mla::launch_decode_pair(tm_q, tm_k32, tm_kv, p, num_workers, st) != cudaSuccess)
+    CUtensorMap tm_po;
+    if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
+    if (mla::launch_decode_pair(tm_q, tm_k32, tm_kv, tm_po, p, num_workers, st) != cudaSuccess)
       return MLA_ERR_CUDA;
   } else {
     if (mla::launch_decode(tm_q, tm_kv, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;

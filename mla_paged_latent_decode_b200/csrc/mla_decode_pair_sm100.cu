@@ -161,10 +161,46 @@ __device__ __forceinline__ void warp_arrive_leader(uint64_t* bar, uint32_t rank,
   }
 }
 
+// Softmax warps: dims 0..383 of the query rows of the piece whose staging
+// entries come next in the K ring, staging slots -> tensor memory (row r in
+// lanes r and r + 64).  Both QK^T warps have finished the previous piece (their
+// Q-empty commit), so no MMA still reads the old rows and neither warp can miss
+// a phase of the Q-ready barrier.
+__device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar,
+                                                volatile int* abort_flag, uint32_t tmem_q, int r,
+                                                uint32_t rank, int lane, int& entries,
+                                                int& qcopies) {
+  const uint8_t* qa = sk + (entries % kKSlots) * kKBytes;
+  const uint8_t* qb = sk + ((entries + 1) % kKSlots) * kKBytes;
+  entries += 2;
+  if (qcopies > 0 && !warp_wait_cluster(&bar[kQEmpty], (qcopies - 1) & 1, abort_flag))
+    return false;
+  if (!warp_wait_cluster(&bar[kQStage], qcopies & 1, abort_flag)) return false;
+  ++qcopies;
+  for (int c = 0; c < kQTmemChunks; ++c) {
+    const uint8_t* rowp = (c < kQStageA ? qa + c * kChunk : qb + (c - kQStageA) * kChunk) + r * 128;
+    uint32_t q[32];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((u ^ (r & 7)) << 4));
+      q[4 * u] = v.x;
+      q[4 * u + 1] = v.y;
+      q[4 * u + 2] = v.z;
+      q[4 * u + 3] = v.w;
+    }
+    tmem_st32(tmem_q + 32 * c, q);
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  warp_arrive_leader(&bar[kQReady], rank, lane);
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k32,
-                       const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
+                       const __grid_constant__ CUtensorMap tm_kv,
+                       const __grid_constant__ CUtensorMap tm_po, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -422,6 +458,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t quarter = static_cast<uint32_t>(32 * warp) << 16;
     int entries = 0, pages = 0, pieces_done = 0, qcopies = 0;
     bool ok = true;
+    bool q_copied_ahead = false;
     for (int pc = 0; pc < npieces && ok; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       const int Lseq = p.seqlens[pz.seq];
@@ -435,39 +472,12 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       float m = -INFINITY, l = 0.f;
 
       if (pz.npg > 0) {
-        // ---- query dims 0..383: staging slots -> tensor memory (row r in lanes r, r + 64).
-        // Both QK^T warps have finished the previous piece (their Q-empty commit),
-        // so no MMA still reads the old rows and neither warp can miss a phase
-        // of the Q-ready barrier.
-        {
-          const uint8_t* qa = sk + (entries % kKSlots) * kKBytes;
-          const uint8_t* qb = sk + ((entries + 1) % kKSlots) * kKBytes;
-          entries += 2;
-          if (qcopies > 0) {
-            ok = warp_wait_cluster(&bar[kQEmpty], (qcopies - 1) & 1, abort_flag);
-            if (!ok) break;
-          }
-          ok = warp_wait_cluster(&bar[kQStage], qcopies & 1, abort_flag);
-          ++qcopies;
+        if (!q_copied_ahead) {
+          ok = copy_query_rows(sk, bar, abort_flag, tmem + quarter + kTmemQ, r, rank, lane, entries,
+                               qcopies);
           if (!ok) break;
-          for (int c = 0; c < kQTmemChunks; ++c) {
-            const uint8_t* rowp =
-                (c < kQStageA ? qa + c * kChunk : qb + (c - kQStageA) * kChunk) + r * 128;
-            uint32_t q[32];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((u ^ (r & 7)) << 4));
-              q[4 * u] = v.x;
-              q[4 * u + 1] = v.y;
-              q[4 * u + 2] = v.z;
-              q[4 * u + 3] = v.w;
-            }
-            tmem_st32(tmem + quarter + kTmemQ + 32 * c, q);
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          warp_arrive_leader(&bar[kQReady], rank, lane);
         }
+        q_copied_ahead = false;
         for (int j = 0; j < pz.npg; ++j) {
           const int g = pages + j, pb = g & 1;
           ok = warp_wait_cluster(&bar[kSFull0 + pb], (g >> 1) & 1, abort_flag);
@@ -515,13 +525,13 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                                    abort_flag);
             if (!ok) break;
             tc_fence_after();
-            for (int cb = 0; cb < 256; cb += 32) {
-              uint32_t o[32];
-              tmem_ld32(tmem + quarter + kTmemO + cb, o);
-              tmem_ld_wait(o);
+            for (int cb = 0; cb < 256; cb += 16) {
+              uint32_t o[16];
+              tmem_ld32x16(tmem + quarter + kTmemO + cb, o);
+              tmem_ld_wait16(o);
 #pragma unroll
-              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-              tmem_st32(tmem + quarter + kTmemO + cb, o);
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32x16(tmem + quarter + kTmemO + cb, o);
             }
             tmem_st_wait();
           }
@@ -549,8 +559,24 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         pages += pz.npg;
         if (!ok) break;
         tc_fence_after();
+        // The next piece with pages gets its query rows now, so that its QK^T
+        // runs while this piece's epilogue drains O.
+        for (int pn = pc + 1; pn < npieces; ++pn) {
+          if (piece_of(md, pn, p.seqlens, p.bt_stride).npg > 0) {
+            ok = copy_query_rows(sk, bar, abort_flag, tmem + quarter + kTmemQ, r, rank, lane,
+                                 entries, qcopies);
+            q_copied_ahead = true;
+            break;
+          }
+        }
+        if (!ok) break;
       }
-      // ---- epilogue: sums of the two row halves, then O / l
+      // ---- epilogue: sums of the two row halves, then O / l.  Each warp owns
+      // rows 32 (warp & 1) .. +31 of this CTA and dv half `th` of each 256-wide
+      // block.  A 32 x 32 block goes TMEM -> registers -> shared memory (the P
+      // buffers, idle until this piece's output is written; 16-byte units
+      // XOR-swizzled by row, so neither side has bank conflicts) -> global
+      // memory, one contiguous row segment per instruction.
       float* lb = sl + (pc & 1) * 128;
       lb[th * 64 + r] = l;
       mbar_arrive(&bar[kLBar]);
@@ -558,10 +584,12 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) break;
       const float lt = l + lb[(th ^ 1) * 64 + r];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const int64_t orow = static_cast<int64_t>(pz.seq) * p.rows + row;
+      float* stg = reinterpret_cast<float*>(sp) + warp * 1024;
+      const int wrow0 = row0 + 32 * (warp & 1);  // sequence row of this warp's lane 0
+      const int64_t orow0 = static_cast<int64_t>(pz.seq) * p.rows + wrow0;
       for (int h = 0; h < 2; ++h) {
-        const int dv0 = 256 * h + 128 * th;
         for (int cb = 0; cb < 128; cb += 32) {
+          const int col = 256 * h + 128 * th + cb;
           uint32_t o[32];
           if (pz.npg > 0) {
             tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb, o);
@@ -570,27 +598,52 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int k = 0; k < 32; ++k) o[k] = 0u;
           }
-          if (!row_ok) continue;
-          if (k_pieces == 1) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + dv0 + cb);
+          // the TMA store of the previous block has read the staging buffer
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+          // row `lane` -> 16-byte unit u ^ (lane & 7) of staging row `lane` (the
+          // layout of a 128-byte-swizzled TMA box of 32 rows x 32 fp32)
+          float4* srow = reinterpret_cast<float4*>(stg + lane * 32);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[8 * u]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
-              dst[u] = v;
+          for (int u = 0; u < 8; ++u)
+            srow[u ^ (lane & 7)] =
+                make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                            __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+          __syncwarp();
+          // row i of the block, one row per instruction: lane l holds column l
+          const int sw_unit = lane >> 2, sw_word = lane & 3;
+          // eight rows at a time: the shared loads issue back to back, then the stores
+          const float* scol = stg + sw_word;
+          if (k_pieces == 1) {
+            for (int i0 = 0; i0 < 32; i0 += 8) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = scol[(i0 + i) * 32 + ((sw_unit ^ i) << 2)];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float w = __shfl_down_sync(0xffffffffu, v[i], 1);
+                if ((lane & 1) == 0 && wrow0 + i0 + i < p.rows)
+                  *reinterpret_cast<uint32_t*>(p.out + (orow0 + i0 + i) * kDv + col + lane) =
+                      pack_bf16x2(v[i], w);
+              }
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * p.rows + row) * kDv + dv0 + cb);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              dst[u] = make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
-                                   __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+            // fp32 partial: one TMA store of the block (rows past the sequence's
+            // query rows fall outside the map and are not written)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_po, stg, col, wrow0, static_cast<int32_t>(slot));
+              tma_store_commit();
+            }
           }
+          __syncwarp();
         }
       }
+      // the P buffers are the staging area: their last store must have read them
+      // before the next piece writes P
+      if (lane == 0) tma_store_wait_read();
+      __syncwarp();
       if (row_ok && th == 0) {
         const float lse = lt > 0.f ? (m + lg2_approx(lt)) * 0.69314718055994531f : -INFINITY;
         if (k_pieces == 1)
@@ -601,6 +654,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   }
 
+  if (warp < kSoftmaxWarps && lane == 0) tma_store_wait_all();  // partial outputs written
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no pair MMA still writes either CTA's tensor memory
@@ -614,8 +668,8 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 }  // namespace
 
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k32,
-                               const CUtensorMap& tm_kv, const DecodeParams& p, int num_workers,
-                               cudaStream_t stream) {
+                               const CUtensorMap& tm_kv, const CUtensorMap& tm_po,
+                               const DecodeParams& p, int num_workers, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -640,7 +694,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k3
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_k32, tm_kv, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_k32, tm_kv, tm_po, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

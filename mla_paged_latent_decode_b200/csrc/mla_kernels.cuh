@@ -55,8 +55,8 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k32,
-                               const CUtensorMap& tm_kv, const DecodeParams& p, int num_workers,
-                               cudaStream_t stream);
+                               const CUtensorMap& tm_kv, const CUtensorMap& tm_po,
+                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t pair_kernel_max_clusters(int* clusters);
 
 }  // namespace mla
