@@ -76,8 +76,15 @@ constexpr int kVBytes = 4 * kChunk;                    // 32768: 64 tokens x 256
 constexpr int kPBytes = kChunk;                        // 64 rows x 64 tokens
 constexpr int kKSlots = 3;
 constexpr int kVSlots = 2;
+// A K-part slot is handed back in three groups of three 64-dim chunks, each as
+// soon as the QK^T MMAs reading it have completed, so the producer refills the
+// start of a slot while the end is still being read.
+constexpr int kKGroups = 3;
+constexpr int kChunksPerGroup = 3;
+constexpr int kKStepsPerGroup = kChunksPerGroup * 4;
 constexpr int kQKSteps = kDqk / 16;                    // 36
 constexpr int kQTmemKSteps = kQTmemChunks * 4;         // 24
+static_assert(kKGroups * kChunksPerGroup == kChunks, "K-part groups cover the page");
 static_assert(kQStageA * kChunk <= kKBytes && (kQTmemChunks - kQStageA) * kChunk <= kKBytes,
               "query staging entries fit a K-part slot");
 
@@ -94,8 +101,9 @@ enum Bar {
   kKFull0 = 0,                                    // leader: K parts of both CTAs
   kVFull0 = kKFull0 + kKSlots,                    // leader: V parts of both CTAs
   kQFull = kVFull0 + kVSlots,                     // leader: Q dims 384..575 of both CTAs
-  kKEmpty0,                                       // both: pair commits (multicast)
-  kVEmpty0 = kKEmpty0 + kKSlots,
+  kKEmpty0,                                       // both: pair commits (multicast),
+                                                  //   [slot][chunk group]
+  kVEmpty0 = kKEmpty0 + kKSlots * kKGroups,
   kQEmpty = kVEmpty0 + kVSlots,
   kSFull0, kSFull1, kPvDone0, kPvDone1, kOFull,   // both: pair commits (multicast)
   kSFree0, kSFree1, kPFull0, kPFull1, kQReady,    // leader: softmax warps of both CTAs
@@ -229,7 +237,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&bar[kKFull0 + s], 1);
-      mbar_init(&bar[kKEmpty0 + s], 1);
+      for (int grp = 0; grp < kKGroups; ++grp) mbar_init(&bar[kKEmpty0 + s * kKGroups + grp], 1);
     }
     for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bar[kVFull0 + s], 1);
@@ -290,11 +298,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         // dims 0..383: two staging entries of the K ring, counted on this CTA's barrier
         for (int e = 0; e < 2; ++e) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
-          if (use > 0) {
-            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
-                                   kWaitLimitNs);
-            if (!ok) break;
-          }
+          for (int grp = 0; grp < kKGroups && use > 0 && ok; ++grp)
+            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot * kKGroups + grp], (use - 1) & 1,
+                                   abort_flag, kWaitLimitNs);
+          if (!ok) break;
           if (e == 0) mbar_arrive_expect_tx(&bar[kQStage], kQTmemChunks * kChunk);
           uint8_t* dst = sk + slot * kKBytes;
           const int c0 = e == 0 ? 0 : kQStageA, c1 = e == 0 ? kQStageA : kQTmemChunks;
@@ -306,19 +313,23 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (!ok) break;
         const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
-        for (int j = 0; j < pz.npg; ++j, ++entries) {
+        for (int j = 0; j < pz.npg && ok; ++j, ++entries) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
-          if (use > 0) {
-            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
-                                   kWaitLimitNs);
-            if (!ok) break;
-          }
           const int page = __ldg(bt + pz.pg0 + j);
-          if (rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
           uint8_t* dst = sk + slot * kKBytes;
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_2d_pair(dst + c * kHalfChunk, &tm_k32, c * 64,
-                             page * kPage + 32 * static_cast<int>(rank), &bar[kKFull0 + slot]);
+          for (int grp = 0; grp < kKGroups; ++grp) {
+            if (use > 0) {
+              ok = mbar_wait_cluster(&bar[kKEmpty0 + slot * kKGroups + grp], (use - 1) & 1,
+                                     abort_flag, kWaitLimitNs);
+              if (!ok) break;
+            }
+            // group 0 released means the QK^T warp has consumed the slot's previous
+            // fill, so the leader's full barrier is in the phase of this entry
+            if (grp == 0 && rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
+            for (int c = grp * kChunksPerGroup; c < (grp + 1) * kChunksPerGroup; ++c)
+              tma_load_2d_pair(dst + c * kHalfChunk, &tm_k32, c * 64,
+                               page * kPage + 32 * static_cast<int>(rank), &bar[kKFull0 + slot]);
+          }
         }
       }
     }
@@ -371,8 +382,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
         tc_fence_after();
         if (parity == 0) {  // both CTAs hold Q in tensor memory: the staging slots are free
-          umma_commit_pair(&bar[kKEmpty0 + stage_a]);
-          umma_commit_pair(&bar[kKEmpty0 + stage_b]);
+          for (int grp = 0; grp < kKGroups; ++grp) {
+            umma_commit_pair(&bar[kKEmpty0 + stage_a * kKGroups + grp]);
+            umma_commit_pair(&bar[kKEmpty0 + stage_b * kKGroups + grp]);
+          }
         }
         for (int j = 0; j < pz.npg && ok; ++j) {
           const int g = pages + j, b = g & 1, entry = entries + j;
@@ -401,9 +414,11 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
               umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
             }
+            if (kk % kKStepsPerGroup == kKStepsPerGroup - 1 && kk != kQKSteps - 1)
+              umma_commit_pair(&bar[kKEmpty0 + slot * kKGroups + kk / kKStepsPerGroup]);
           }
           umma_commit_pair(&bar[kSFull0 + b]);
-          umma_commit_pair(&bar[kKEmpty0 + slot]);
+          umma_commit_pair(&bar[kKEmpty0 + slot * kKGroups + kKGroups - 1]);
         }
         if (!ok) break;
         umma_commit_pair(&bar[kQEmpty]);  // this warp's reads of Q for the piece are done
