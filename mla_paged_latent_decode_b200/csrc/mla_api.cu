@@ -76,6 +76,25 @@ bool make_partial_map(CUtensorMap* map, float* base, uint64_t rows, uint64_t slo
   return r == CUDA_SUCCESS;
 }
 
+// The cache viewed as 3-D {64 dims, rows, 9 chunks} (strides: a row is 1152
+// bytes, a chunk 128): one box of box_rows rows x box_chunks 64-dim chunks lands
+// in shared memory chunk after chunk, each chunk box_rows x 128 bytes with
+// 128-byte swizzle, which is the layout the MMA descriptors read.  One TMA
+// instruction then moves several chunks.
+bool make_chunk_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows,
+                    uint32_t box_chunks) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(mla::kDqk / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk) * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Query rows up to 64 per sequence run on single CTAs (one 64-row block); more
@@ -181,10 +200,9 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
 
   const int rows = s_q * h_q;
-  CUtensorMap tm_q, tm_kv;
+  CUtensorMap tm_q;
   if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
-  if (!make_row_map(&tm_kv, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage))
-    return MLA_ERR_CUDA;
+  const uint64_t cache_rows = static_cast<uint64_t>(num_blocks) * mla::kPage;
 
   const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
   float* part_o = static_cast<float*>(workspace);
@@ -212,15 +230,19 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (uses_pairs(s_q, h_q)) {
-    CUtensorMap tm_k32;
-    if (!make_row_map(&tm_k32, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage, 32))
-      return MLA_ERR_CUDA;
+    // K part: 32 token rows x 3 chunks per box; V part: 64 rows x 2 chunks
+    CUtensorMap tm_kpart, tm_vpart;
+    if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, 3)) return MLA_ERR_CUDA;
+    if (!make_chunk_map(&tm_vpart, kcache, cache_rows, 64, 2)) return MLA_ERR_CUDA;
     CUtensorMap tm_po;
     if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
-    if (mla::launch_decode_pair(tm_q, tm_k32, tm_kv, tm_po, p, num_workers, st) != cudaSuccess)
+    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vpart, tm_po, p, num_workers, st) != cudaSuccess)
       return MLA_ERR_CUDA;
   } else {
-    if (mla::launch_decode(tm_q, tm_kv, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
+    // a whole page (64 rows x 9 chunks) per box
+    CUtensorMap tm_page;
+    if (!make_chunk_map(&tm_page, kcache, cache_rows, 64, mla::kDqk / 64)) return MLA_ERR_CUDA;
+    if (mla::launch_decode(tm_q, tm_page, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
   }
 
   mla::CombineParams c{};

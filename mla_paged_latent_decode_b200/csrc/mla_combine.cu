@@ -8,9 +8,10 @@
 // pages give no such step (their decode kernel is described only as
 // "optimized for variable-length" serving, "OpenSourceWeek Day 1: FlashMLA").
 //
-// One warp per query row: each lane owns 16 of the 512 values as 4 float4
-// (coalesced 512-byte warp loads), and the weights are recomputed per lane
-// from the piece lses.
+// One warp per query row.  Lane s holds piece s's lse (pieces in groups of 32),
+// so the maximum, the sum and every weight come from shuffles after a single
+// load; each lane owns 16 of the 512 values as 4 float4 (coalesced 512-byte
+// warp loads), and the loads of several pieces are in flight together.
 #include "mla_kernels.cuh"
 
 namespace mla {
@@ -52,18 +53,26 @@ mla_combine_kernel(const CombineParams p) {
   float4 acc[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < k; ++s) {
-    const float ls = lse_col[static_cast<int64_t>(s) * p.rows];
-    const float w = ls == -INFINITY ? 0.f : __expf(ls - lse);
-    const float4* src = reinterpret_cast<const float4*>(
-        p.part_o + ((static_cast<int64_t>(base) + s) * p.rows + row) * kDv);
+  const float4* part = reinterpret_cast<const float4*>(
+      p.part_o + (static_cast<int64_t>(base) * p.rows + row) * kDv) + lane;
+  const int64_t piece_stride = static_cast<int64_t>(p.rows) * kDv / 4;  // in float4
+  for (int s0 = 0; s0 < k; s0 += 32) {
+    // lane s: weight of piece s0 + s (the lse was read above, so this hits in cache)
+    const float ls = s0 + lane < k ? lse_col[static_cast<int64_t>(s0 + lane) * p.rows] : -INFINITY;
+    const float my_w = ls == -INFINITY ? 0.f : __expf(ls - lse);
+    const int n = k - s0 < 32 ? k - s0 : 32;
+#pragma unroll 2
+    for (int s = 0; s < n; ++s) {
+      const float w = __shfl_sync(0xffffffffu, my_w, s);
+      const float4* src = part + (s0 + s) * piece_stride;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 v = src[lane + 32 * u];
-      acc[u].x += w * v.x;
-      acc[u].y += w * v.y;
-      acc[u].z += w * v.z;
-      acc[u].w += w * v.w;
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = src[32 * u];
+        acc[u].x += w * v.x;
+        acc[u].y += w * v.y;
+        acc[u].z += w * v.z;
+        acc[u].w += w * v.w;
+      }
     }
   }
 #pragma unroll

@@ -206,8 +206,8 @@ __device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar
 
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k32,
-                       const __grid_constant__ CUtensorMap tm_kv,
+                       const __grid_constant__ CUtensorMap tm_kpart,
+                       const __grid_constant__ CUtensorMap tm_vpart,
                        const __grid_constant__ CUtensorMap tm_po, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -277,7 +277,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------ query rows + K parts
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k32);
+      prefetch_tensormap(&tm_kpart);
       int entries = 0, qloads = 0;
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
@@ -326,9 +326,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             // group 0 released means the QK^T warp has consumed the slot's previous
             // fill, so the leader's full barrier is in the phase of this entry
             if (grp == 0 && rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
-            for (int c = grp * kChunksPerGroup; c < (grp + 1) * kChunksPerGroup; ++c)
-              tma_load_2d_pair(dst + c * kHalfChunk, &tm_k32, c * 64,
-                               page * kPage + 32 * static_cast<int>(rank), &bar[kKFull0 + slot]);
+            // one box: 32 token rows x the group's 3 chunks
+            tma_load_3d_pair(dst + grp * kChunksPerGroup * kHalfChunk, &tm_kpart, 0,
+                             page * kPage + 32 * static_cast<int>(rank), grp * kChunksPerGroup,
+                             &bar[kKFull0 + slot]);
           }
         }
       }
@@ -336,7 +337,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == kTmaVWarp) {
     // ------------------------------------------------------------ V parts
     if (lane == 0) {
-      prefetch_tensormap(&tm_kv);
+      prefetch_tensormap(&tm_vpart);
       int pages = 0;
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
@@ -353,12 +354,11 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int page = __ldg(bt + pz.pg0 + j);
           if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kVBytes);
           uint8_t* dst = sv + slot * kVBytes;
-          // sub-chunk 2h + e holds dv block 4h + 2 rank + e (64 dv each)
+          // sub-chunks 2h, 2h + 1 hold dv blocks 4h + 2 rank, +1 (64 dv each): one box
+          // of 64 rows x 2 chunks per h
           for (int h = 0; h < 2; ++h)
-            for (int e = 0; e < 2; ++e)
-              tma_load_2d_pair(dst + (2 * h + e) * kChunk, &tm_kv,
-                               64 * (4 * h + 2 * static_cast<int>(rank) + e), page * kPage,
-                               &bar[kVFull0 + slot]);
+            tma_load_3d_pair(dst + 2 * h * kChunk, &tm_vpart, 0, page * kPage,
+                             4 * h + 2 * static_cast<int>(rank), &bar[kVFull0 + slot]);
         }
       }
     }
@@ -682,8 +682,8 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 }  // namespace
 
-cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k32,
-                               const CUtensorMap& tm_kv, const CUtensorMap& tm_po,
+cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
+                               const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
                                const DecodeParams& p, int num_workers, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
@@ -709,7 +709,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k3
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_k32, tm_kv, tm_po, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vpart, tm_po, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -125,7 +125,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_kv, const DecodeParams p) {
+                        const __grid_constant__ CUtensorMap tm_page, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -176,7 +176,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_kv);
+      prefetch_tensormap(&tm_page);
       int entries = 0;
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
@@ -198,9 +198,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
           } else {
             const int page = __ldg(bt + pz.pg0 + e);
-            for (int c = 0; c < kChunks; ++c)
-              tma_load_2d(dst + c * kChunkBytes, &tm_kv, c * 64, page * kPage,
-                          &bar[kFull0 + stage]);
+            tma_load_3d(dst, &tm_page, 0, page * kPage, 0, &bar[kFull0 + stage]);
           }
           ++entries;
         }
@@ -514,7 +512,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 }  // namespace
 
-cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
@@ -529,7 +527,7 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
   dim3 grid(num_workers, row_blocks);
-  mla_decode_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_kv, p);
+  mla_decode_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_page, p);
   return cudaGetLastError();
 }
 

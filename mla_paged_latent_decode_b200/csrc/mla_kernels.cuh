@@ -50,12 +50,12 @@ struct CombineParams {
 // Launchers (return cudaGetLastError() of their launch).
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int32_t* tile_md,
                             int32_t* num_splits, cudaStream_t stream);
-cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
+cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
-cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_k32,
-                               const CUtensorMap& tm_kv, const CUtensorMap& tm_po,
+cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
+                               const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
                                const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t pair_kernel_max_clusters(int* clusters);
 
