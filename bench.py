@@ -42,8 +42,11 @@ from mla_paged_latent_decode_b200 import synth  # noqa: E402
 METRIC = "MLA decode TB/s and TFLOPS on one B200 (bf16, paged KV), % of roofline"
 UNIT = "TB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dsv3_decode_traffic.md")
-DECODE_SRC = os.path.join(ROOT, "mla_paged_latent_decode_b200", "csrc", "mla_decode_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "mla_decode_pair_kernel_dsv3_decode_traffic.md")
+CSRC = os.path.join(ROOT, "mla_paged_latent_decode_b200", "csrc")
+# more than 64 query rows per sequence run on CTA pairs, fewer on single CTAs
+PAIR_SRC = os.path.join(CSRC, "mla_decode_pair_sm100.cu")
+SINGLE_SRC = os.path.join(CSRC, "mla_decode_sm100.cu")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -56,8 +59,13 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def decode_source_sha():
-    with open(DECODE_SRC, "rb") as f:
+def decode_source(workload: str) -> str:
+    w = synth.WORKLOADS[workload]
+    return PAIR_SRC if w.s_q * w.h_q > 64 else SINGLE_SRC
+
+
+def decode_source_sha(workload: str):
+    with open(decode_source(workload), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
@@ -72,7 +80,7 @@ def recorded_traffic(workload: str):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 fields[k.strip()] = v.strip()
-    if fields.get("decode_kernel_source_sha256_16") != decode_source_sha():
+    if fields.get("decode_kernel_source_sha256_16") != decode_source_sha(workload):
         return None
     try:
         return int(fields["dram_bytes_per_launch"])
