@@ -38,6 +38,38 @@ def test_forced_splits(cuda_device, num_workers):
     full_parity(inp, cuda_device, num_workers=num_workers)
 
 
+@pytest.mark.parametrize("num_workers", [1, 2, 5, 37, 74, 300])
+def test_forced_splits_pairs(cuda_device, num_workers):
+    # more than 64 query rows run on CTA pairs: two 128-row blocks per worker,
+    # every split plan
+    w = synth.custom_workload(3, 2, 128, [700, 5, 1100], causal=True)
+    inp = synth.make_inputs(w, seed=8)
+    full_parity(inp, cuda_device, num_workers=num_workers)
+
+
+def test_pair_split_reuses_workspace(cuda_device):
+    # leftovers of an earlier call on the same workspace, or arbitrary bytes in
+    # it, must not change the result
+    from mla_paged_latent_decode_b200 import binding
+    w = synth.custom_workload(4, 1, 128, [3000, 64, 1900, 700])
+    inp = synth.make_inputs(w, seed=12)
+    q, kc, bt, sl = (t.to(cuda_device) for t in (inp.q, inp.kcache, inp.block_table, inp.cache_seqlens))
+    md, ns = binding.get_mla_metadata(sl, inp.h_q, inp.s_q, 40)
+    assert int(ns[-1].item()) > inp.batch  # some sequence is split
+    ws = torch.full((binding.workspace_size(inp.batch, inp.s_q, inp.h_q, 40),), 0xFF,
+                    dtype=torch.uint8, device=cuda_device)
+    outs = []
+    for _ in range(3):
+        out, lse = binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal,
+                                              workspace=ws)
+        torch.cuda.synchronize(cuda_device)
+        outs.append((out.float().cpu().numpy(), lse.cpu().numpy()))
+    for o, l in outs[1:]:
+        np.testing.assert_array_equal(o, outs[0][0])
+        np.testing.assert_array_equal(l, outs[0][1])
+    full_parity(inp, cuda_device, num_workers=40)
+
+
 def test_empty_and_degenerate_sequences(cuda_device):
     # L = 0 (nothing visible), L = 1 < s_q (first query empty under causal), exact pages
     w = synth.custom_workload(5, 2, 16, [0, 1, 64, 128, 2], causal=True)
