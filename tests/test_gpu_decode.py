@@ -47,6 +47,17 @@ def test_forced_splits_pairs(cuda_device, num_workers):
     full_parity(inp, cuda_device, num_workers=num_workers)
 
 
+@pytest.mark.parametrize("s_q,h_q,causal", [(3, 32, True), (1, 96, False), (4, 128, True),
+                                             (2, 96, True), (1, 65, False)])
+def test_pair_row_blocks(cuda_device, s_q, h_q, causal):
+    # query-row counts on the CTA-pair path: a second CTA with some or no valid
+    # rows (96, 65 rows), several 128-row blocks per worker (192, 384, 512 rows)
+    w = synth.custom_workload(3, s_q, h_q, [900, 3, 200], causal=causal)
+    inp = synth.make_inputs(w, seed=20 + s_q * h_q)
+    full_parity(inp, cuda_device)
+    full_parity(inp, cuda_device, num_workers=7)
+
+
 def test_pair_split_reuses_workspace(cuda_device):
     # leftovers of an earlier call on the same workspace, or arbitrary bytes in
     # it, must not change the result
