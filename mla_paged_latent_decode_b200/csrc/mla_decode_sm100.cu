@@ -135,6 +135,9 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
+  // Launched as a programmatic dependent of the scheduler kernel: its CTAs may
+  // start while the scheduler runs, and read the metadata only after this wait.
+  grid_dependency_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int worker = blockIdx.x, rb = blockIdx.y;
   const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
@@ -526,8 +529,18 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
     configured[dev] = true;
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
-  dim3 grid(num_workers, row_blocks);
-  mla_decode_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_page, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_workers, row_blocks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel, tm_q, tm_page, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@
 // sequence); each thread owns a contiguous chunk of sequences and writes the
 // worker rows whose first or last item falls in one of them.
 #include "mla_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -54,6 +55,8 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
                     int32_t* __restrict__ tile_md, int32_t* __restrict__ num_splits) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t total_units, total_pieces;
+  grid_dependency_wait();     // the lengths may come from the previous kernel
+  grid_launch_dependents();   // the decode may be scheduled; it waits for this grid
   const int tid = threadIdx.x;
   const int chunk = (batch + blockDim.x - 1) / blockDim.x;
   const int i0 = min(batch, tid * chunk), i1 = min(batch, i0 + chunk);
@@ -125,8 +128,18 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int32_t* tile_md,
                             int32_t* num_splits, cudaStream_t stream) {
-  mla_metadata_kernel<<<1, kMdThreads, 0, stream>>>(seqlens, batch, num_workers, tile_md,
-                                                    num_splits);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kMdThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, seqlens, batch, num_workers,
+                                     tile_md, num_splits);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -150,6 +150,17 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Programmatic dependent launch.  wait: block until the grids this one depends
+// on have completed and their writes are visible (nothing to wait for when the
+// grid was launched without the attribute).  launch_dependents: let the next
+// grid in the stream be scheduled now; it still waits for this grid before it
+// reads anything this grid writes.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
