@@ -14,7 +14,10 @@
 namespace mla {
 namespace {
 
-constexpr int kMdThreads = 1024;
+constexpr int kMdThreads = 256;
+// Up to this many workers, the rows are assembled in shared memory and written
+// out once; beyond it they are assembled in place in global memory.
+constexpr int kSmemWorkers = 1024;
 
 // Exclusive scan of one int64 per thread across the block; also returns the total.
 __device__ int64_t block_exclusive_scan(int64_t v, int64_t* warp_sums, int64_t* total) {
@@ -52,9 +55,12 @@ __device__ __forceinline__ int64_t items_of(int32_t L) {
 
 __global__ void __launch_bounds__(kMdThreads)
 mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_workers,
-                    int32_t* __restrict__ tile_md, int32_t* __restrict__ num_splits) {
+                    int32_t* __restrict__ tile_md_global, int32_t* __restrict__ num_splits) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t total_units, total_pieces;
+  __shared__ int32_t srows[kSmemWorkers * kMdStride];
+  const bool in_smem = num_workers <= kSmemWorkers;
+  int32_t* tile_md = in_smem ? srows : tile_md_global;
   grid_dependency_wait();     // the lengths may come from the previous kernel
   grid_launch_dependents();   // the decode may be scheduled; it waits for this grid
   const int tid = threadIdx.x;
@@ -62,6 +68,7 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
   const int i0 = min(batch, tid * chunk), i1 = min(batch, i0 + chunk);
 
   for (int k = tid; k < num_workers * kMdStride; k += blockDim.x) tile_md[k] = 0;
+  if (in_smem) __syncthreads();
 
   // pass 1: unit starts
   int64_t my_units = 0;
@@ -121,6 +128,10 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
       // rows were written above exactly for those workers
       if (row[3] > 0) row[5] = row[2] - row[0] + 1;
     }
+  }
+  if (in_smem) {  // one coalesced pass out
+    __syncthreads();
+    for (int k = tid; k < num_workers * kMdStride; k += blockDim.x) tile_md_global[k] = srows[k];
   }
 }
 
