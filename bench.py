@@ -10,8 +10,10 @@ through the C ABI.  The default workload is DeepSeek-V3-shaped decode: batch
 64, s_q 1, 128 heads, every sequence 4096 tokens, 64-token pages shuffled in
 the block table, q and cache ~ N(0, 1) in bf16, scale 1/sqrt(192).
 
-Timing: W untimed warm-up steps, then exactly K steps, each preceded by a
-256 MB device write that flushes L2 (outside the step's event pair); every
+Timing: W untimed warm-up steps, then exactly K steps, each preceded by an L2
+flush outside the step's event pair: a 256 MB device write, then a read of the
+same 256 MB, which evicts the write's dirty lines so that their write-back is
+not charged to the step (the step starts on a cold, clean L2); every
 step is timed with CUDA events on the launching stream; the K timed steps are
 bracketed by a barrier and a device synchronise on both sides; the reported
 time is the maximum over ranks.  With N > 1 every rank runs the same workload
@@ -160,7 +162,9 @@ def workload_config(inp, extra=None):
            "h_q": inp.h_q, "d_qk": 576, "dv": 512, "page": 64,
            "total_cached_tokens": int(inp.cache_seqlens.sum()), "causal": bool(inp.causal),
            "scale": inp.scale, "seed": inp.seed,
-           "l2": "flushed before every timed step by a 256 MB device write"}
+           "l2": "flushed before every timed step (outside its events) by a 256 MB device "
+                 "write followed by a read of the same 256 MB, so the step starts on a cold L2 "
+                 "holding no dirty lines"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -305,7 +309,14 @@ def run_cuda(args, rank, local, world):
                      device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def flush_l2(k):
+        # The write replaces every line of L2; the read that follows evicts the
+        # write's dirty lines (their write-back happens here, not in the step).
+        flush.fill_(k & 0xFF)
+        torch.sum(flush.view(torch.int32), dim=0, dtype=torch.int64, out=flush_sum)
 
     def step():
         md, ns = binding.get_mla_metadata(sl, h_q, s_q, num_workers)
@@ -327,7 +338,7 @@ def run_cuda(args, rank, local, world):
     with ClockSampler(local) as clocks:
         t_wall0 = time.perf_counter()
         for k in range(args.steps):
-            flush.fill_(k & 0xFF)
+            flush_l2(k)
             e0, ev_mid, e1 = events[k]
             e0.record(stream)
             step()
@@ -376,7 +387,7 @@ def run_cuda(args, rank, local, world):
         barrier(world, dev)
         torch.cuda.synchronize(dev)
         for k in range(n_e2e):
-            flush.fill_(k & 0xFF)
+            flush_l2(k)
             a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             e2e_step()
