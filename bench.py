@@ -14,10 +14,16 @@ Timing: W untimed warm-up steps, then exactly K steps, each preceded by an L2
 flush outside the step's event pair: a 256 MB device write, then a read of the
 same 256 MB, which evicts the write's dirty lines so that their write-back is
 not charged to the step (the step starts on a cold, clean L2); every
-step is timed with CUDA events on the launching stream; the K timed steps are
+step is timed with CUDA events on the launching stream, with nothing between
+the scheduler and decode calls (the decode kernel starts, as a programmatic
+dependent, while the scheduler finishes); the K timed steps are
 bracketed by a barrier and a device synchronise on both sides; the reported
 time is the maximum over ranks.  With N > 1 every rank runs the same workload
 on its own GPU (independent replicas; the decode has no cross-GPU exchange).
+After the timed steps, up to 200 more steps with an event between the two
+calls give the scheduler's time and the decode call's (decode kernel + split
+combine), which the roofline uses; there the decode starts only after the
+scheduler has finished.
 
 `--impl reference` times the fp64 CPU oracle on this host instead (bounded
 samples of the same workload), printing the same JSON line with
@@ -309,37 +315,42 @@ def run_cuda(args, rank, local, world):
                      device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
-    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
+    flush_max = torch.empty((), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def flush_l2(k):
         # The write replaces every line of L2; the read that follows evicts the
         # write's dirty lines (their write-back happens here, not in the step).
         flush.fill_(k & 0xFF)
-        torch.sum(flush.view(torch.int32), dim=0, dtype=torch.int64, out=flush_sum)
+        torch.amax(flush.view(torch.int32), dim=0, out=flush_max)
 
-    def step():
-        md, ns = binding.get_mla_metadata(sl, h_q, s_q, num_workers)
-        ev_mid.record(stream)
+    def metadata():
+        return binding.get_mla_metadata(sl, h_q, s_q, num_workers)
+
+    def decode_call(md, ns):
         binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal, out=out,
                                    lse=lse, workspace=ws, device_status=status)
 
+    def step():
+        # nothing between the two calls: the decode kernel is a programmatic
+        # dependent of the scheduler kernel and starts while it finishes
+        decode_call(*metadata())
+
     for _ in range(args.warmup):
-        ev_mid = torch.cuda.Event(enable_timing=True)
         step()
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during warm-up")
 
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-               torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         t_wall0 = time.perf_counter()
         for k in range(args.steps):
             flush_l2(k)
-            e0, ev_mid, e1 = events[k]
+            e0, e1 = events[k]
             e0.record(stream)
             step()
             e1.record(stream)
@@ -347,9 +358,29 @@ def run_cuda(args, rank, local, world):
         t_wall = time.perf_counter() - t_wall0
     barrier(world, dev)
     torch.cuda.synchronize(dev)
-    step_ms = [e0.elapsed_time(e1) for e0, _, e1 in events]
-    decode_ms = [m.elapsed_time(e1) for _, m, e1 in events]
-    meta_ms = [e0.elapsed_time(m) for e0, m, _ in events]
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in events]
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during timing")
+
+    # The two calls timed apart (an event between them, so here the decode kernel
+    # starts only once the scheduler has finished): the scheduler's time, and the
+    # decode call's (decode kernel + split combine) for the roofline.
+    n_split = max(3, min(args.steps, 200))
+    split_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+                    for _ in range(n_split)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    for k in range(n_split):
+        flush_l2(k)
+        e0, em, e1 = split_events[k]
+        e0.record(stream)
+        md_k, ns_k = metadata()
+        em.record(stream)
+        decode_call(md_k, ns_k)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    decode_ms = [m.elapsed_time(e1) for _, m, e1 in split_events]
+    meta_ms = [e0.elapsed_time(m) for e0, m, _ in split_events]
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during timing")
 
