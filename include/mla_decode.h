@@ -57,7 +57,8 @@ typedef enum {
 #define MLA_HEAD_DIM_V 512      /* value = first 512 dims of the same row */
 #define MLA_PAGE_SIZE 64        /* tokens per cache page */
 #define MLA_MD_STRIDE 8         /* int32 per worker in tile_md */
-#define MLA_SPLIT_PIECE_COST 2  /* fixed cost of one piece, in pages (partition rule) */
+#define MLA_SPLIT_PIECE_COST_CTA 2   /* per-sequence cost in pages, s_q * h_q <= 64 (partition rule) */
+#define MLA_SPLIT_PIECE_COST_PAIR 7  /* per-sequence cost in pages, s_q * h_q > 64 (partition rule) */
 #define MLA_ROWS_PER_CTA 64     /* query rows (s_q * h_q, flattened) per decode CTA */
 #define MLA_STATIC_SCRATCH_BYTES ((size_t)48 << 20) /* see mla_decode_kvcache_static_scratch */
 
@@ -83,10 +84,14 @@ int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_st
  * Day 1: FlashMLA", opening paragraph; "DeepSeek merilis open source FlashMLA",
  * release bullets) and give no partition rule.  The rule used here:
  *   n_i = ceil(L_i / 64) pages; items_i = max(n_i, 1) (an empty sequence owns one
- *   item so that its zero output is written); sequence i costs
- *   MLA_SPLIT_PIECE_COST + items_i units, laid end to end from unit start_i, with
- *   item j at unit start_i + MLA_SPLIT_PIECE_COST + j; cap = ceil(total / W);
- *   the item at unit u goes to worker u / cap.
+ *   item so that its zero output is written); sequence i costs P + items_i units,
+ *   laid end to end from unit start_i, with item j at unit start_i + P + j;
+ *   cap = ceil(total / W); the item at unit u goes to worker u / cap.
+ *   P = MLA_SPLIT_PIECE_COST_CTA when s_q * h_q <= 64 (one CTA per worker) and
+ *   MLA_SPLIT_PIECE_COST_PAIR otherwise (CTA pairs): roughly what starting and
+ *   finishing a piece costs that kernel, in page-loop time.  It was set by
+ *   measurement: on a CTA pair, a piece boundary stalls the page loop for its
+ *   epilogue (fp32 or bf16 output of 128 rows x 512), about 8 pages' time.
  * Each worker thus owns a contiguous run of items.  A sequence whose items fall
  * to k workers has k pieces (splits), merged by log-sum-exp in the decode call.
  *
@@ -99,7 +104,7 @@ int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_st
  *                pieces per sequence (num_splits[0] = 0).
  * num_workers:   >= 1; normally the value from mla_metadata_shape.  The same
  *                value must be passed to mla_decode_kvcache.
- * h_q, s_q:      checked only (> 0); the rule itself depends on lengths and W.
+ * h_q, s_q:      > 0; s_q * h_q selects P (the decode kernel is chosen the same way).
  * One CTA; integer only; no host synchronisation.  batch <= 65536.
  */
 int mla_get_metadata(const int32_t* cache_seqlens, int batch, int h_q, int s_q,

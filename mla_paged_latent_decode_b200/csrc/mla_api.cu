@@ -162,8 +162,9 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int h_q, int s_q,
   if (batch < 1 || batch > 65536 || h_q < 1 || s_q < 1 || num_workers < 1 ||
       num_workers > (1 << 20))
     return MLA_ERR_INVALID_ARG;
-  cudaError_t e = mla::launch_metadata(cache_seqlens, batch, num_workers, tile_md, num_splits,
-                                       static_cast<cudaStream_t>(stream));
+  const int piece_cost = uses_pairs(s_q, h_q) ? MLA_SPLIT_PIECE_COST_PAIR : MLA_SPLIT_PIECE_COST_CTA;
+  cudaError_t e = mla::launch_metadata(cache_seqlens, batch, num_workers, piece_cost, tile_md,
+                                       num_splits, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

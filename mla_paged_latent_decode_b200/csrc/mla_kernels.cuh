@@ -16,7 +16,6 @@ constexpr int kDqk = MLA_HEAD_DIM_QK;     // 576
 constexpr int kDv = MLA_HEAD_DIM_V;       // 512
 constexpr int kRowsPerCta = MLA_ROWS_PER_CTA;
 constexpr int kMdStride = MLA_MD_STRIDE;
-constexpr int kPieceCost = MLA_SPLIT_PIECE_COST;
 
 // Bounded device waits give up after this long (then report MLA_ERR_DEVICE_TIMEOUT).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -48,8 +47,8 @@ struct CombineParams {
 };
 
 // Launchers (return cudaGetLastError() of their launch).
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int32_t* tile_md,
-                            int32_t* num_splits, cudaStream_t stream);
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,
+                            int32_t* tile_md, int32_t* num_splits, cudaStream_t stream);
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);

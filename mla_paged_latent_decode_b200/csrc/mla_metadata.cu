@@ -1,9 +1,10 @@
 // mla_metadata.cu -- the length-balanced split-KV tile scheduler.
 //
 // Rule (stated in include/mla_decode.h, mla_get_metadata): sequence i owns
-// items_i = max(ceil(L_i / 64), 1) items and costs kPieceCost + items_i units;
-// laid end to end, its item j sits at unit start_i + kPieceCost + j, and the
-// item at unit u belongs to worker u / cap with cap = ceil(total / W).
+// items_i = max(ceil(L_i / 64), 1) items and costs P + items_i units, P the
+// per-sequence cost of the decode kernel the rows select; laid end to end, its
+// item j sits at unit start_i + P + j, and the item at unit u belongs to worker
+// u / cap with cap = ceil(total / W).
 //
 // One CTA computes it with two block-wide scans (unit starts, then pieces per
 // sequence); each thread owns a contiguous chunk of sequences and writes the
@@ -54,7 +55,7 @@ __device__ __forceinline__ int64_t items_of(int32_t L) {
 }
 
 __global__ void __launch_bounds__(kMdThreads)
-mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_workers,
+mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_workers, int piece_cost,
                     int32_t* __restrict__ tile_md_global, int32_t* __restrict__ num_splits) {
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t total_units, total_pieces;
@@ -72,7 +73,7 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
 
   // pass 1: unit starts
   int64_t my_units = 0;
-  for (int i = i0; i < i1; ++i) my_units += kPieceCost + items_of(seqlens[i]);
+  for (int i = i0; i < i1; ++i) my_units += piece_cost + items_of(seqlens[i]);
   const int64_t my_start = block_exclusive_scan(my_units, warp_sums, &total_units);
   __syncthreads();
   const int64_t total = total_units;
@@ -84,7 +85,7 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
     int64_t s = my_start;
     for (int i = i0; i < i1; ++i) {
       const int64_t n = items_of(seqlens[i]);
-      const int64_t f = s + kPieceCost, g = f + n - 1;
+      const int64_t f = s + piece_cost, g = f + n - 1;
       my_pieces += g / cap - f / cap + 1;
       s = g + 1;
     }
@@ -95,11 +96,11 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
     int64_t s = my_start, pc = my_first_piece;
     for (int i = i0; i < i1; ++i) {
       const int64_t n = items_of(seqlens[i]);
-      const int64_t f = s + kPieceCost, g = f + n - 1;
+      const int64_t f = s + piece_cost, g = f + n - 1;
       const int64_t w_first = f / cap, w_last = g / cap;
       pc += w_last - w_first + 1;
       num_splits[i + 1] = static_cast<int32_t>(pc);
-      const int64_t next_first_item = g + 1 + kPieceCost;  // first item unit of sequence i+1
+      const int64_t next_first_item = g + 1 + piece_cost;  // first item unit of sequence i+1
       for (int64_t w = w_first; w <= w_last; ++w) {
         int32_t* row = tile_md + w * kMdStride;
         const int64_t lo = w * cap, hi = lo + cap;
@@ -137,8 +138,8 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
 
 }  // namespace
 
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int32_t* tile_md,
-                            int32_t* num_splits, cudaStream_t stream) {
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,
+                            int32_t* tile_md, int32_t* num_splits, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kMdThreads);
@@ -149,7 +150,7 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, mla_metadata_kernel, seqlens, batch, num_workers,
-                                     tile_md, num_splits);
+                                     piece_cost, tile_md, num_splits);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -9,9 +9,12 @@ Python loops so that the GPU's metadata can be compared with it bit for bit:
   n_i     = ceil(L_i / 64) pages of sequence i
   items_i = max(n_i, 1)        (an empty sequence still owns one item: its
                                  output, zeros and lse = -inf, must be written)
-  every sequence costs PIECE_COST + items_i units; laid end to end, sequence i
-  starts at unit start_i and its item j sits at unit start_i + PIECE_COST + j.
+  every sequence costs P + items_i units; laid end to end, sequence i starts
+  at unit start_i and its item j sits at unit start_i + P + j.
   cap     = ceil(total / W);  the item at unit u belongs to worker u // cap.
+  P       = PIECE_COST_CTA (2) when s_q * h_q <= 64 query rows run on one CTA
+            per worker, PIECE_COST_PAIR (7) when they run on CTA pairs; the
+            header states both as the library's tuned constants.
 
 A worker therefore owns one contiguous run of items, which may begin or end
 inside a sequence.  A sequence spread over k workers yields k pieces ("splits")
@@ -25,15 +28,23 @@ num_splits[i + 1] - num_splits[i] is the number of pieces of sequence i.
 from __future__ import annotations
 
 PAGE = 64
-PIECE_COST = 2
+PIECE_COST_CTA = 2
+PIECE_COST_PAIR = 7
+ROWS_PER_CTA = 64
 MD_STRIDE = 8
 
 
-def split_plan(seqlens, num_workers: int):
+def piece_cost_for(s_q: int, h_q: int) -> int:
+    """The per-sequence cost P the rule uses for s_q * h_q query rows."""
+    return PIECE_COST_CTA if s_q * h_q <= ROWS_PER_CTA else PIECE_COST_PAIR
+
+
+def split_plan(seqlens, num_workers: int, piece_cost: int):
     """Returns (tile_md as a list of num_workers rows of 8 ints, num_splits list of b+1)."""
     lens = [int(v) for v in seqlens]
     W = int(num_workers)
-    assert W >= 1
+    P = int(piece_cost)
+    assert W >= 1 and P >= 0
     items = []
     for L in lens:
         n = (L + PAGE - 1) // PAGE if L > 0 else 0
@@ -42,14 +53,14 @@ def split_plan(seqlens, num_workers: int):
     total = 0
     for it in items:
         starts.append(total)
-        total += PIECE_COST + it
+        total += P + it
     cap = max(1, -(-total // W))
 
     # which worker owns each item, written out item by item
     owner = {}
     for i, it in enumerate(items):
         for j in range(it):
-            owner[(i, j)] = (starts[i] + PIECE_COST + j) // cap
+            owner[(i, j)] = (starts[i] + P + j) // cap
 
     md = [[0] * MD_STRIDE for _ in range(W)]
     pieces_of_seq = [0] * len(lens)

@@ -39,7 +39,8 @@ def expected_workers(dev, s_q, h_q):
 
 
 def check_metadata(inp, res, num_workers):
-    md, ns = scheduler.split_plan(inp.cache_seqlens.tolist(), num_workers)
+    md, ns = scheduler.split_plan(inp.cache_seqlens.tolist(), num_workers,
+                                  scheduler.piece_cost_for(inp.s_q, inp.h_q))
     np.testing.assert_array_equal(res["tile_md"].numpy(), np.asarray(md, dtype=np.int32))
     np.testing.assert_array_equal(res["num_splits"].numpy(), np.asarray(ns, dtype=np.int32))
 

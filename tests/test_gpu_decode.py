@@ -160,14 +160,18 @@ def test_metadata_bit_exact_many_shapes(cuda_device):
         lens = torch.randint(0, 20000, (b,), generator=g, dtype=torch.int32)
         lens[::5] = 0
         sl = lens.to(cuda_device)
-        for W in (1, 5, 74, 148, 2000):
-            tile_md, num_splits = binding.get_mla_metadata(sl, 16, 1, W)
-            torch.cuda.synchronize()
-            res = {"tile_md": tile_md.cpu(), "num_splits": num_splits.cpu()}
+        # both per-sequence costs: single-CTA rows (16 heads) and CTA-pair rows (128)
+        for h_q in (16, 128) if b <= 1000 else (16,):
+            for W in (1, 5, 74, 148, 2000):
+                tile_md, num_splits = binding.get_mla_metadata(sl, h_q, 1, W)
+                torch.cuda.synchronize()
+                res = {"tile_md": tile_md.cpu(), "num_splits": num_splits.cpu()}
 
-            class _I:
-                cache_seqlens = lens
-            check_metadata(_I, res, W)
+                class _I:
+                    cache_seqlens = lens
+                    s_q = 1
+                _I.h_q = h_q
+                check_metadata(_I, res, W)
 
 
 def test_host_validation_rejects_bad_arguments(cuda_device):

@@ -7,15 +7,17 @@ import itertools
 
 import pytest
 
-from oracle.scheduler import PAGE, PIECE_COST, split_plan
+from oracle.scheduler import PAGE, PIECE_COST_CTA, PIECE_COST_PAIR, piece_cost_for, split_plan
+
+COSTS = (PIECE_COST_CTA, PIECE_COST_PAIR)
 
 
 def items_of(L):
     return max((L + PAGE - 1) // PAGE, 1)
 
 
-def check_plan(lens, W):
-    md, ns = split_plan(lens, W)
+def check_plan(lens, W, P):
+    md, ns = split_plan(lens, W, P)
     b = len(lens)
     assert len(md) == W and len(ns) == b + 1 and ns[0] == 0
     # every item of every sequence is covered exactly once, workers in order
@@ -48,7 +50,7 @@ def check_plan(lens, W):
             expect = md[w][4] if md[w][0] == i else 0
             assert s == expect
     # balance: no worker owns more than cap items
-    total = sum(PIECE_COST + items_of(L) for L in lens)
+    total = sum(P + items_of(L) for L in lens)
     cap = -(-total // W)
     for w in range(W):
         assert sum(1 for v in seen.values() if v == w) <= cap
@@ -57,43 +59,67 @@ def check_plan(lens, W):
     return md, ns
 
 
-def test_single_worker_takes_everything():
-    md, ns = check_plan([37, 130, 0], 1)
+def test_cost_follows_the_kernel_the_rows_select():
+    # up to 64 query rows run on one CTA per worker, more on CTA pairs
+    assert piece_cost_for(1, 16) == piece_cost_for(1, 64) == piece_cost_for(4, 16) == PIECE_COST_CTA
+    assert piece_cost_for(1, 65) == piece_cost_for(1, 128) == piece_cost_for(2, 128) == PIECE_COST_PAIR
+
+
+@pytest.mark.parametrize("P", COSTS)
+def test_single_worker_takes_everything(P):
+    md, ns = check_plan([37, 130, 0], 1, P)
     assert md[0][:6] == [0, 0, 2, 1, 0, 3]
     assert ns == [0, 1, 2, 3]
 
 
-def test_one_sequence_per_worker_when_costs_align():
-    # 4 sequences of 6 pages each, cost 8 units each, 4 workers: one each, no splits
-    md, ns = check_plan([6 * 64] * 4, 4)
+@pytest.mark.parametrize("P", COSTS)
+def test_one_sequence_per_worker_when_costs_align(P):
+    # 4 sequences of 6 pages each, P + 6 units each, 4 workers: one each, no splits
+    md, ns = check_plan([6 * 64] * 4, 4, P)
     assert ns == [0, 1, 2, 3, 4]
     assert [r[:6] for r in md] == [[i, 0, i, 6, 0, 1] for i in range(4)]
 
 
-def test_long_sequence_is_split_across_workers():
-    md, ns = check_plan([32768] * 15 + [1], 74)
+def test_cost_moves_pages_off_workers_that_start_sequences():
+    # 3 sequences of 10 pages, 2 workers.  P = 2: 36 units, cap 18, worker 0
+    # takes units 0..17 = sequence 0 (2 + 10) and units 12..17 of sequence 1,
+    # i.e. its cost and 4 pages.  P = 7: 51 units, cap 26, worker 0 takes
+    # sequence 0 (7 + 10) and units 17..25 of sequence 1, its cost and 2 pages.
+    md, ns = check_plan([640] * 3, 2, 2)
+    assert md[0][:6] == [0, 0, 1, 4, 0, 2]
+    md, ns = check_plan([640] * 3, 2, 7)
+    assert md[0][:6] == [0, 0, 1, 2, 0, 2]
+    assert md[1][:6] == [1, 2, 2, 10, 1, 2]
+
+
+@pytest.mark.parametrize("P", COSTS)
+def test_long_sequence_is_split_across_workers(P):
+    md, ns = check_plan([32768] * 15 + [1], 74, P)
     assert ns[-1] > 16                  # the long sequences are cut
     assert ns[16] - ns[15] == 1         # the one-token sequence is whole
 
 
-def test_more_workers_than_items():
-    md, ns = check_plan([37, 130], 148)
+@pytest.mark.parametrize("P", COSTS)
+def test_more_workers_than_items(P):
+    md, ns = check_plan([37, 130], 148, P)
     assert sum(1 for r in md if r[5] > 0) == 4   # one worker per page
     assert ns == [0, 1, 4]
 
 
+@pytest.mark.parametrize("P", COSTS)
 @pytest.mark.parametrize("W", [1, 2, 3, 5, 7])
-def test_brute_force_small(W):
+def test_brute_force_small(W, P):
     lengths = [0, 1, 63, 64, 65, 128, 129, 300]
     for b in (1, 2, 3):
         for lens in itertools.product(lengths, repeat=b):
-            check_plan(list(lens), W)
+            check_plan(list(lens), W, P)
 
 
-def test_realistic_shapes():
+@pytest.mark.parametrize("P", COSTS)
+def test_realistic_shapes(P):
     import torch
     g = torch.Generator().manual_seed(0)
     for W in (37, 74, 148):
         lens = torch.randint(1, 8193, (128,), generator=g).tolist()
-        check_plan(lens, W)
-        check_plan([4096] * 64, W)
+        check_plan(lens, W, P)
+        check_plan([4096] * 64, W, P)
