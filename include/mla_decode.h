@@ -92,6 +92,10 @@ int mla_metadata_shape(int batch, int h_q, int s_q, int* num_workers, int* md_st
  *   finishing a piece costs that kernel, in page-loop time.  It was set by
  *   measurement: on a CTA pair, a piece boundary stalls the page loop for its
  *   epilogue (fp32 or bf16 output of 128 rows x 512), about 8 pages' time.
+ *   Exception (whole sequences): when batch <= W and no sequence costs more than
+ *   cap + 2 P units, worker i takes all items of sequence i (i < batch) and the
+ *   other workers are idle: a split would save at most about 2 P pages of the
+ *   longest worker's time, less than its piece boundaries and the merge cost.
  * Each worker thus owns a contiguous run of items.  A sequence whose items fall
  * to k workers has k pieces (splits), merged by log-sum-exp in the decode call.
  *

@@ -4,7 +4,8 @@
 // items_i = max(ceil(L_i / 64), 1) items and costs P + items_i units, P the
 // per-sequence cost of the decode kernel the rows select; laid end to end, its
 // item j sits at unit start_i + P + j, and the item at unit u belongs to worker
-// u / cap with cap = ceil(total / W).
+// u / cap with cap = ceil(total / W).  Exception: with batch <= W and every
+// sequence costing at most cap + 2 P units, worker i takes sequence i whole.
 //
 // One CTA computes it with two block-wide scans (unit starts, then pieces per
 // sequence); each thread owns a contiguous chunk of sequences and writes the
@@ -49,6 +50,22 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* warp_sums, int64_t* 
   return r;
 }
 
+// Maximum of one int64 per thread across the block.
+__device__ int64_t block_max(int64_t v, int64_t* warp_vals) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const int64_t n = __shfl_xor_sync(0xffffffffu, v, o);
+    v = n > v ? n : v;
+  }
+  if (lane == 0) warp_vals[warp] = v;
+  __syncthreads();
+  int64_t m = warp_vals[0];
+  for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = warp_vals[w] > m ? warp_vals[w] : m;
+  __syncthreads();
+  return m;
+}
+
 __device__ __forceinline__ int64_t items_of(int32_t L) {
   const int64_t n = L > 0 ? (static_cast<int64_t>(L) + kPage - 1) / kPage : 0;
   return n > 0 ? n : 1;
@@ -78,6 +95,34 @@ mla_metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int num_work
   __syncthreads();
   const int64_t total = total_units;
   const int64_t cap = total > 0 ? (total + num_workers - 1) / num_workers : 1;
+
+  // Whole sequences: with no more sequences than workers, and no sequence
+  // costing more than cap + 2 P units, worker i takes sequence i and nothing is
+  // split (no partial outputs, nothing to merge).
+  int64_t my_max = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int64_t u = piece_cost + items_of(seqlens[i]);
+    my_max = u > my_max ? u : my_max;
+  }
+  const int64_t umax = block_max(my_max, warp_sums);
+  if (batch <= num_workers && umax <= cap + 2 * static_cast<int64_t>(piece_cost)) {
+    if (tid == 0) num_splits[0] = 0;
+    for (int i = i0; i < i1; ++i) {
+      int32_t* row = tile_md + static_cast<int64_t>(i) * kMdStride;
+      row[0] = i;
+      row[1] = 0;
+      row[2] = i;
+      row[3] = static_cast<int32_t>(items_of(seqlens[i]));
+      row[4] = 0;
+      row[5] = 1;
+      num_splits[i + 1] = i + 1;
+    }
+    if (in_smem) {
+      __syncthreads();
+      for (int k = tid; k < num_workers * kMdStride; k += blockDim.x) tile_md_global[k] = srows[k];
+    }
+    return;
+  }
 
   // pass 2: pieces per sequence, and the worker rows that begin or end here
   int64_t my_pieces = 0;

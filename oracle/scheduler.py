@@ -15,6 +15,8 @@ Python loops so that the GPU's metadata can be compared with it bit for bit:
   P       = PIECE_COST_CTA (2) when s_q * h_q <= 64 query rows run on one CTA
             per worker, PIECE_COST_PAIR (7) when they run on CTA pairs; the
             header states both as the library's tuned constants.
+  Exception: if b <= W and every sequence costs at most cap + 2 P units, the
+  sequences stay whole: worker i takes every item of sequence i (i < b).
 
 A worker therefore owns one contiguous run of items, which may begin or end
 inside a sequence.  A sequence spread over k workers yields k pieces ("splits")
@@ -55,6 +57,12 @@ def split_plan(seqlens, num_workers: int, piece_cost: int):
         starts.append(total)
         total += P + it
     cap = max(1, -(-total // W))
+
+    if len(lens) <= W and max(P + it for it in items) <= cap + 2 * P:
+        md = [[0] * MD_STRIDE for _ in range(W)]
+        for i, it in enumerate(items):
+            md[i] = [i, 0, i, it, 0, 1, 0, 0]
+        return md, list(range(len(lens) + 1))
 
     # which worker owns each item, written out item by item
     owner = {}

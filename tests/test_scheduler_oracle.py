@@ -49,11 +49,18 @@ def check_plan(lens, W, P):
         for s, (w, lo, hi) in enumerate(pieces[i]):
             expect = md[w][4] if md[w][0] == i else 0
             assert s == expect
-    # balance: no worker owns more than cap items
+    # balance: no worker owns more than cap items; with sequences kept whole
+    # (b <= W and no sequence above cap + 2P units) one sequence per worker
     total = sum(P + items_of(L) for L in lens)
     cap = -(-total // W)
-    for w in range(W):
-        assert sum(1 for v in seen.values() if v == w) <= cap
+    whole = b <= W and max(P + items_of(L) for L in lens) <= cap + 2 * P
+    if whole:
+        assert ns == list(range(b + 1))
+        for w in range(W):
+            assert md[w][:6] == ([w, 0, w, items_of(lens[w]), 0, 1] if w < b else [0] * 6)
+    else:
+        for w in range(W):
+            assert sum(1 for v in seen.values() if v == w) <= cap
     # pieces beyond one per sequence come only from worker boundaries
     assert ns[-1] <= b + W - 1
     return md, ns
@@ -92,6 +99,29 @@ def test_cost_moves_pages_off_workers_that_start_sequences():
     assert md[1][:6] == [1, 2, 2, 10, 1, 2]
 
 
+def test_uniform_long_sequences_stay_whole():
+    # 64 sequences of 64 pages on 74 workers.  P = 7: 71 units each, cap 62,
+    # 71 <= 62 + 14, so one worker per sequence and no splits.  P = 2: 66 units,
+    # cap 58, 66 > 58 + 4, so the linear rule splits them.
+    md, ns = check_plan([4096] * 64, 74, 7)
+    assert ns == list(range(65)) and sum(1 for r in md if r[5]) == 64
+    md, ns = check_plan([4096] * 64, 74, 2)
+    assert ns[-1] > 64
+
+
+def test_whole_sequence_threshold():
+    # two workers, P = 7.  30 + 2 pages: 37 + 9 = 46 units, cap 23, the longest
+    # is 37 = cap + 14: whole.  32 + 2 pages: 39 + 9 = 48 units, cap 24, 39 > 38:
+    # split by the linear rule.
+    md, ns = check_plan([30 * 64, 2 * 64], 2, 7)
+    assert ns == [0, 1, 2] and md[0][:6] == [0, 0, 0, 30, 0, 1] and md[1][:6] == [1, 0, 1, 2, 0, 1]
+    md, ns = check_plan([32 * 64, 2 * 64], 2, 7)
+    assert ns == [0, 2, 3]
+    # more sequences than workers: the linear rule (worker 1 takes sequences 1 and 2)
+    md, ns = check_plan([64] * 3, 2, 7)
+    assert ns == [0, 1, 2, 3] and md[1][:6] == [1, 0, 2, 1, 0, 2]
+
+
 @pytest.mark.parametrize("P", COSTS)
 def test_long_sequence_is_split_across_workers(P):
     md, ns = check_plan([32768] * 15 + [1], 74, P)
@@ -101,9 +131,14 @@ def test_long_sequence_is_split_across_workers(P):
 
 @pytest.mark.parametrize("P", COSTS)
 def test_more_workers_than_items(P):
+    # 1 + 3 pages on 148 workers: cap 1 and the longer sequence costs P + 3 <=
+    # 1 + 2P units, so both stay whole
     md, ns = check_plan([37, 130], 148, P)
-    assert sum(1 for r in md if r[5] > 0) == 4   # one worker per page
-    assert ns == [0, 1, 4]
+    assert ns == [0, 1, 2] and sum(1 for r in md if r[5] > 0) == 2
+    # 1 + 20 pages: P + 20 > 1 + 2P, so the linear rule gives one worker per page
+    md, ns = check_plan([37, 20 * 64], 148, P)
+    assert sum(1 for r in md if r[5] > 0) == 21
+    assert ns == [0, 1, 21]
 
 
 @pytest.mark.parametrize("P", COSTS)
