@@ -16,6 +16,7 @@
 // round trip to memory.  out = acc / sum and lse = m + ln(sum) at the end,
 // which equals the formula above.
 #include "mla_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -27,10 +28,16 @@ constexpr int kPiecesPerRound = 4;
 
 __global__ void __launch_bounds__(kCombineThreads)
 mla_combine_kernel(const CombineParams p) {
+  // Launched as a programmatic dependent of the decode kernel.  The piece
+  // counts come from the scheduler, which finished before any decode CTA got
+  // past its own dependency wait, so they are read before this grid's wait: a
+  // sequence with one piece (its output written by the decode) needs nothing,
+  // and its blocks leave without waiting for the decode to finish.
   const int seq = blockIdx.x;
   const int base = p.num_splits[seq];
   const int k = p.num_splits[seq + 1] - base;
   if (k <= 1) return;
+  grid_dependency_wait();  // the decode's partial outputs are complete and visible
   const int t = blockIdx.y * kCombineThreads + threadIdx.x;
   const int row = t / kRowThreads, c = t % kRowThreads;
   if (row >= p.rows) return;
@@ -101,8 +108,17 @@ mla_combine_kernel(const CombineParams p) {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   // x: sequences (any batch size); y: blocks of four query rows (rows <= 65536)
-  dim3 grid(p.batch, (p.rows * kRowThreads + kCombineThreads - 1) / kCombineThreads);
-  mla_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.batch, (p.rows * kRowThreads + kCombineThreads - 1) / kCombineThreads);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mla_combine_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
