@@ -138,7 +138,7 @@ size_t mla_workspace_size(int batch, int s_q, int h_q, int dv, int num_workers);
  *               cache_seqlens (the same stream order makes them ready).
  * workspace:    device scratch of at least mla_workspace_size(...) bytes,
  *               256-byte aligned; contents need not be initialised.
- * out:          device bf16 [batch, s_q, h_q, 512], written.
+ * out:          device bf16 [batch, s_q, h_q, 512], 16-byte aligned, written.
  * lse:          device fp32 [batch, h_q, s_q], written (natural log).
  * device_status: device int32, or NULL; receives MLA_ERR_DEVICE_* on a device
  *               condition (never reset by the library: the caller zeroes it).

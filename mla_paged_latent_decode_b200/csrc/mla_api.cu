@@ -76,6 +76,24 @@ bool make_partial_map(CUtensorMap* map, float* base, uint64_t rows, uint64_t slo
   return r == CUDA_SUCCESS;
 }
 
+// The bf16 output [batch, rows, 512] written in boxes of 32 rows x 64 columns
+// (128 bytes per row) with 128-byte swizzle; the row extent clips boxes that run
+// past a sequence's rows.
+bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t batch) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDv), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDv) * 2,
+                           static_cast<cuuint64_t>(mla::kDv) * 2 * rows};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // The cache viewed as 3-D {64 dims, rows, 9 chunks} (strides: a row is 1152
 // bytes, a chunk 128): one box of box_rows rows x box_chunks 64-dim chunks lands
 // in shared memory chunk after chunk, each chunk box_rows x 128 bytes with
@@ -235,9 +253,12 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
     CUtensorMap tm_kpart, tm_vpart;
     if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, 3)) return MLA_ERR_CUDA;
     if (!make_chunk_map(&tm_vpart, kcache, cache_rows, 64, 2)) return MLA_ERR_CUDA;
-    CUtensorMap tm_po;
+    CUtensorMap tm_po, tm_out;
     if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
-    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vpart, tm_po, p, num_workers, st) != cudaSuccess)
+    if (!make_out_map(&tm_out, out, static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)))
+      return MLA_ERR_CUDA;
+    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vpart, tm_po, tm_out, p, num_workers, st) !=
+        cudaSuccess)
       return MLA_ERR_CUDA;
   } else {
     // a whole page (64 rows x 9 chunks) per box

@@ -208,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kpart,
                        const __grid_constant__ CUtensorMap tm_vpart,
-                       const __grid_constant__ CUtensorMap tm_po, const DecodeParams p) {
+                       const __grid_constant__ CUtensorMap tm_po,
+                       const __grid_constant__ CUtensorMap tm_out, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -591,10 +592,12 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       // ---- epilogue: sums of the two row halves, then O / l.  Each warp owns
       // rows 32 (warp & 1) .. +31 of this CTA and dv half `th` of each 256-wide
-      // block.  A 32 x 32 block goes TMEM -> registers -> shared memory (the P
-      // buffers, idle until this piece's output is written; 16-byte units
-      // XOR-swizzled by row, so neither side has bank conflicts) -> global
-      // memory, one contiguous row segment per instruction.
+      // block.  Blocks go TMEM -> registers -> shared memory (the P buffers,
+      // idle until this piece's output is written; 16-byte units XOR-swizzled by
+      // row, so neither side has bank conflicts) -> global memory: by TMA store
+      // for fp32 partials and for the bf16 output of the CTA's last piece, by
+      // the load/store units (one contiguous row segment per instruction) for
+      // the bf16 output of an earlier piece.
       float* lb = sl + (pc & 1) * 128;
       lb[th * 64 + r] = l;
       mbar_arrive(&bar[kLBar]);
@@ -604,58 +607,103 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       float* stg = reinterpret_cast<float*>(sp) + warp * 1024;
       const int wrow0 = row0 + 32 * (warp & 1);  // sequence row of this warp's lane 0
-      const int64_t orow0 = static_cast<int64_t>(pz.seq) * p.rows + wrow0;
-      for (int h = 0; h < 2; ++h) {
-        for (int cb = 0; cb < 128; cb += 32) {
-          const int col = 256 * h + 128 * th + cb;
-          uint32_t o[32];
-          if (pz.npg > 0) {
-            tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb, o);
-            tmem_ld_wait(o);
-          } else {
+      if (k_pieces == 1 && pc == npieces - 1) {
+        // bf16 output of this CTA's last piece: blocks of 32 rows x 64 dv columns
+        // (128 bytes per row), one TMA store each (rows past the sequence's query
+        // rows fall outside the map and are not written).  Only the last piece:
+        // earlier, TMA stores would queue with the next piece's page loads.
+        for (int h = 0; h < 2; ++h) {
+          for (int cb = 0; cb < 128; cb += 64) {
+            const int col = 256 * h + 128 * th + cb;
+            uint32_t w[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = 0u;
-          }
-          // the TMA store of the previous block has read the staging buffer
-          if (lane == 0) tma_store_wait_read();
-          __syncwarp();
-          // row `lane` -> 16-byte unit u ^ (lane & 7) of staging row `lane` (the
-          // layout of a 128-byte-swizzled TMA box of 32 rows x 32 fp32)
-          float4* srow = reinterpret_cast<float4*>(stg + lane * 32);
+            for (int half = 0; half < 2; ++half) {
+              uint32_t o[32];
+              if (pz.npg > 0) {
+                tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb + 32 * half, o);
+                tmem_ld_wait(o);
+              } else {
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            srow[u ^ (lane & 7)] =
-                make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
-                            __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
-          __syncwarp();
-          // row i of the block, one row per instruction: lane l holds column l
-          const int sw_unit = lane >> 2, sw_word = lane & 3;
-          // eight rows at a time: the shared loads issue back to back, then the stores
-          const float* scol = stg + sw_word;
-          if (k_pieces == 1) {
-            for (int i0 = 0; i0 < 32; i0 += 8) {
-              float v[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = scol[(i0 + i) * 32 + ((sw_unit ^ i) << 2)];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float w = __shfl_down_sync(0xffffffffu, v[i], 1);
-                if ((lane & 1) == 0 && wrow0 + i0 + i < p.rows)
-                  *reinterpret_cast<uint32_t*>(p.out + (orow0 + i0 + i) * kDv + col + lane) =
-                      pack_bf16x2(v[i], w);
+                for (int k = 0; k < 32; ++k) o[k] = 0u;
               }
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                w[16 * half + k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv,
+                                               __uint_as_float(o[2 * k + 1]) * inv);
             }
-          } else {
-            // fp32 partial: one TMA store of the block (rows past the sequence's
-            // query rows fall outside the map and are not written)
+            // the TMA store of the previous block has read the staging buffer
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+            // row `lane` -> 16-byte unit u ^ (lane & 7) of staging row `lane` (the
+            // layout of a 128-byte-swizzled TMA box of 32 rows x 64 bf16)
+            uint4* srow = reinterpret_cast<uint4*>(stg + lane * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              srow[u ^ (lane & 7)] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&tm_po, stg, col, wrow0, static_cast<int32_t>(slot));
+              tma_store_3d(&tm_out, stg, col, wrow0, pz.seq);
               tma_store_commit();
             }
+            __syncwarp();
           }
-          __syncwarp();
+        }
+      } else {
+        const int64_t orow0 = static_cast<int64_t>(pz.seq) * p.rows + wrow0;
+        for (int h = 0; h < 2; ++h) {
+          for (int cb = 0; cb < 128; cb += 32) {
+            const int col = 256 * h + 128 * th + cb;
+            uint32_t o[32];
+            if (pz.npg > 0) {
+              tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb, o);
+              tmem_ld_wait(o);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = 0u;
+            }
+            // the TMA store of the previous block has read the staging buffer
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+            // row `lane` -> 16-byte unit u ^ (lane & 7) of staging row `lane` (the
+            // layout of a 128-byte-swizzled TMA box of 32 rows x 32 fp32)
+            float4* srow = reinterpret_cast<float4*>(stg + lane * 32);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              srow[u ^ (lane & 7)] = make_float4(
+                  __uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                  __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+            __syncwarp();
+            if (k_pieces == 1) {
+              // bf16 output of an earlier piece, through the load/store units: row
+              // i of the block per instruction, lane l holding column l; eight
+              // rows at a time, the shared loads back to back, then the stores
+              const int sw_unit = lane >> 2, sw_word = lane & 3;
+              const float* scol = stg + sw_word;
+              for (int i0 = 0; i0 < 32; i0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = scol[(i0 + i) * 32 + ((sw_unit ^ i) << 2)];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float w = __shfl_down_sync(0xffffffffu, v[i], 1);
+                  if ((lane & 1) == 0 && wrow0 + i0 + i < p.rows)
+                    *reinterpret_cast<uint32_t*>(p.out + (orow0 + i0 + i) * kDv + col + lane) =
+                        pack_bf16x2(v[i], w);
+                }
+              }
+            } else {
+              // fp32 partial: one TMA store of the block (rows past the sequence's
+              // query rows fall outside the map and are not written)
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tm_po, stg, col, wrow0, static_cast<int32_t>(slot));
+                tma_store_commit();
+              }
+            }
+            __syncwarp();
+          }
         }
       }
       // the P buffers are the staging area: their last store must have read them
@@ -687,7 +735,8 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
                                const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
-                               const DecodeParams& p, int num_workers, cudaStream_t stream) {
+                               const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
+                               cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -714,7 +763,7 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vpart, tm_po, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vpart, tm_po, tm_out, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

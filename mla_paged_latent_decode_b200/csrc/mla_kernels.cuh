@@ -55,7 +55,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
                                const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
-                               const DecodeParams& p, int num_workers, cudaStream_t stream);
+                               const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
+                               cudaStream_t stream);
 cudaError_t pair_kernel_max_clusters(int* clusters);
 
 }  // namespace mla
