@@ -10,7 +10,9 @@ through the C ABI.  The default workload is DeepSeek-V3-shaped decode: batch
 64, s_q 1, 128 heads, every sequence 4096 tokens, 64-token pages shuffled in
 the block table, q and cache ~ N(0, 1) in bf16, scale 1/sqrt(192).
 
-Timing: W untimed warm-up steps, then exactly K steps, each preceded by an L2
+Timing: W untimed warm-up steps, then exactly K steps, each a replay of a CUDA
+graph of the step captured after the warm-up (the same three kernels, no host
+work inside the events; e2e below runs eagerly), each preceded by an L2
 flush outside the step's event pair: a 256 MB device write, then a read of the
 same 256 MB, which evicts the write's dirty lines so that their write-back is
 not charged to the step (the step starts on a cold, clean L2); every
@@ -20,10 +22,10 @@ dependent, while the scheduler finishes); the K timed steps are
 bracketed by a barrier and a device synchronise on both sides; the reported
 time is the maximum over ranks.  With N > 1 every rank runs the same workload
 on its own GPU (independent replicas; the decode has no cross-GPU exchange).
-After the timed steps, up to 200 more steps with an event between the two
-calls give the scheduler's time and the decode call's (decode kernel + split
-combine), which the roofline uses; there the decode starts only after the
-scheduler has finished.
+After the timed steps, up to 200 more steps, replaying graphs of the two calls
+with an event between them, give the scheduler's time and the decode call's
+(decode kernel + split combine), which the roofline uses; there the decode
+starts only after the scheduler has finished.
 
 `--impl reference` times the fp64 CPU oracle on this host instead (bounded
 samples of the same workload), printing the same JSON line with
@@ -170,7 +172,10 @@ def workload_config(inp, extra=None):
            "scale": inp.scale, "seed": inp.seed,
            "l2": "flushed before every timed step (outside its events) by a 256 MB device "
                  "write followed by a read of the same 256 MB, so the step starts on a cold L2 "
-                 "holding no dirty lines"}
+                 "holding no dirty lines",
+           "timing": "each timed step replays a CUDA graph of the step (scheduler, decode and "
+                     "combine kernels) captured after the warm-up; e2e runs eagerly through the "
+                     "public API"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -342,6 +347,30 @@ def run_cuda(args, rank, local, world):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during warm-up")
 
+    # The timed steps replay CUDA graphs of the calls (captured once, after the
+    # warm-up), as a serving loop would: the same three kernels per step, with
+    # no host work (argument checks, tensor-map encoding, launches) inside the
+    # events.  g_step is the whole step; g_meta and g_call are the two calls
+    # captured apart, for the split below.
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g_step, g_meta, g_call = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
+    with torch.cuda.graph(g_meta):
+        md_g, ns_g = metadata()
+    with torch.cuda.graph(g_call):
+        decode_call(md_g, ns_g)
+    for k in range(3):
+        flush_l2(k)
+        g_step.replay()
+    torch.cuda.synchronize(dev)
+
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     barrier(world, dev)
@@ -352,7 +381,7 @@ def run_cuda(args, rank, local, world):
             flush_l2(k)
             e0, e1 = events[k]
             e0.record(stream)
-            step()
+            g_step.replay()
             e1.record(stream)
         torch.cuda.synchronize(dev)
         t_wall = time.perf_counter() - t_wall0
@@ -374,11 +403,12 @@ def run_cuda(args, rank, local, world):
         flush_l2(k)
         e0, em, e1 = split_events[k]
         e0.record(stream)
-        md_k, ns_k = metadata()
+        g_meta.replay()
         em.record(stream)
-        decode_call(md_k, ns_k)
+        g_call.replay()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    del g_step, g_meta, g_call
     decode_ms = [m.elapsed_time(e1) for _, m, e1 in split_events]
     meta_ms = [e0.elapsed_time(m) for e0, m, _ in split_events]
     if int(status.item()) != 0:
