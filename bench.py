@@ -464,6 +464,8 @@ def run_cuda(args, rank, local, world):
                "note": "q, block_table and cache_seqlens copied in, out and lse copied back each "
                        "step; the latent cache stays resident in HBM as in serving"}
 
+    append = None if args.no_append else measure_append(inp, dev, stream, flush_l2)
+
     if rank != 0:
         return None
     peaks, peak_kind = load_peaks()
@@ -502,6 +504,10 @@ def run_cuda(args, rank, local, world):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if append is not None:
+        for case in append.values():
+            case["frac_of_hbm_peak"] = case["gb_s"] / peaks["hbm_gbs"]
+        line["append"] = append
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         sub, dt, what = oracle_sample(inp, args.cpu_seconds)
@@ -510,6 +516,71 @@ def run_cuda(args, rank, local, world):
             "value": tbs, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
             "sample": f"{what}, {dt:.1f} s", "tflops": tfl}
     return line
+
+
+def measure_append(inp, dev, stream, flush_l2, calls=50):
+    """Time mla_append_latent (the latent-cache append with page allocation) on
+    the workload's batch: every sequence sits at a page boundary, so every call
+    takes one new page per sequence (the costliest decode step), for s_new = s_q
+    (one decode step) and for s_new = 1024 (a chunk, large enough to show the
+    copy's bandwidth).  Each call replays a CUDA graph of the append after the
+    cache state has been restored and L2 flushed, outside its events.
+    Algorithmic bytes: the new rows read and written (1152 B each), plus 16 B
+    per sequence of lengths, block-table entries and popped free-stack slots."""
+    from mla_paged_latent_decode_b200 import binding
+    b = inp.batch
+    res = {}
+    for name, s_new in (("decode_step", inp.s_q), ("chunk_1024", 1024)):
+        new_pages = -(-s_new // 64)
+        pool = b * (1 + new_pages)
+        gen = torch.Generator().manual_seed(1)
+        kc = torch.randn((pool, 64, 576), generator=gen).to(torch.bfloat16).to(dev)
+        rows = torch.randn((b, s_new, 576), generator=gen).to(torch.bfloat16).to(dev)
+        perm = torch.randperm(pool, generator=gen).to(torch.int32)
+        bt0 = torch.zeros((b, 1 + new_pages), dtype=torch.int32)
+        bt0[:, 0] = perm[:b]
+        free0 = perm[b:].contiguous()
+        bt0, free0 = bt0.to(dev), free0.to(dev)
+        sl0 = torch.full((b,), 64, dtype=torch.int32, device=dev)
+        fc0 = torch.tensor([pool - b], dtype=torch.int32, device=dev)
+        bt, sl, free, fc = bt0.clone(), sl0.clone(), free0.clone(), fc0.clone()
+        status = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+        def restore():
+            bt.copy_(bt0)
+            sl.copy_(sl0)
+            fc.copy_(fc0)
+
+        def call():
+            binding.append_latent(rows, kc, bt, sl, free, fc, status)
+
+        for _ in range(3):
+            restore()
+            call()
+        torch.cuda.synchronize(dev)
+        if int(status.item()) != 0 or int(fc.item()) != 0 or int(sl[0].item()) != 64 + s_new:
+            raise RuntimeError(f"append check failed: status {int(status.item())}")
+        graph = torch.cuda.CUDAGraph()
+        restore()
+        with torch.cuda.graph(graph):
+            call()
+        evs = []
+        for k in range(calls):
+            restore()
+            flush_l2(k)
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            z.record(stream)
+            evs.append((a, z))
+        torch.cuda.synchronize(dev)
+        del graph
+        us = statistics.median(a.elapsed_time(z) for a, z in evs) * 1e3
+        nbytes = 2 * b * s_new * 1152 + 16 * b
+        res[name] = {"s_new": s_new, "batch": b, "us": us, "bytes": nbytes,
+                     "gb_s": nbytes / (us * 1e-6) / 1e9, "launches": 2,
+                     "note": "every sequence takes a new page; L2 flushed before each call"}
+    return res
 
 
 def main():
@@ -521,6 +592,8 @@ def main():
     ap.add_argument("--workload", default="dsv3_decode", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
+    ap.add_argument("--no-append", action="store_true",
+                    help="skip timing the latent-cache append")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="approximate oracle time for the cpu_baseline sample")
     args = ap.parse_args()

@@ -50,7 +50,9 @@ typedef enum {
     MLA_ERR_CUDA = 3,           /* a CUDA runtime call failed */
     MLA_ERR_DEVICE_TIMEOUT = 4, /* a device-side wait gave up (device_status only) */
     MLA_ERR_DEVICE_CHECK = 5,   /* a device-side bounds check failed (device_status only) */
-    MLA_ERR_SCRATCH_LIMIT = 6   /* workspace would exceed MLA_STATIC_SCRATCH_BYTES */
+    MLA_ERR_SCRATCH_LIMIT = 6,  /* workspace would exceed MLA_STATIC_SCRATCH_BYTES */
+    MLA_ERR_NO_FREE_PAGES = 7   /* free-page stack too short for an append, or too
+                                   full for a release (device_status only) */
 } mla_status;
 
 #define MLA_HEAD_DIM_QK 576     /* 512 latent + 64 rope dims per row */
@@ -186,6 +188,74 @@ int mla_decode_kvcache_static_scratch(const void* q, const void* kcache, int64_t
                                       const int32_t* tile_md, const int32_t* num_splits,
                                       int num_workers, void* out, float* lse,
                                       int32_t* device_status, void* stream);
+
+/*
+ * mla_append_latent -- add s_new tokens' latent rows to every sequence of the
+ * paged cache, taking new 64-token pages from a free-page stack.
+ *
+ * After each decoding step the newest token's cached state joins the cache for
+ * later steps ("DeepSeek #OpenSourceWeek Day 1: Launch of FlashMLA", "How KV
+ * Caching Works?"); in MLA that state is one latent row per token ("How MLA
+ * Optimizes Memory Usage").  Pages are allocated on demand, like OS virtual
+ * memory, so a sequence grows in 64-token increments ("FlashMLA:
+ * Revolutionizing Efficient Decoding...", section 4.3.2).  The pages give no
+ * allocation order; the rule here:
+ *   - sequence i with L_i = cache_seqlens[i] tokens holds ceil(L_i / 64) pages;
+ *     it needs ceil((L_i + s_new) / 64) - ceil(L_i / 64) new ones;
+ *   - free pages are the stack free_pages[0 : *free_count]; pages are popped
+ *     from the top, sequence after sequence in batch order, page after page
+ *     within a sequence, into block_table[i][ceil(L_i / 64) ...];
+ *   - row k of sequence i becomes token L_i + k: it is copied to row
+ *     (L_i + k) % 64 of page block_table[i][(L_i + k) / 64];
+ *   - then cache_seqlens[i] += s_new and *free_count drops by the pages taken.
+ * Call it before the decode of the step that attends to the new tokens.
+ *
+ * rows:          device bf16 [batch, s_new, 576], 16-byte aligned (read).
+ * s_new:         tokens added to every sequence, 1 .. 65536.
+ * kcache:        device bf16 [num_blocks, 64, 576], 16-byte aligned (written).
+ * block_table:   device int32 [batch, bt_stride] (entries past each sequence's
+ *                pages are written as pages are taken).
+ * cache_seqlens: device int32 [batch] (read, then grown).
+ * free_pages:    device int32 [free_capacity]: the free-page stack (read).
+ * free_count:    device int32 [1]: pages on the stack, 0 .. free_capacity
+ *                (read, then lowered).
+ * device_status: device int32 or NULL, as for mla_decode_kvcache.
+ * The request is checked as a whole on the device.  If any L_i is negative,
+ * ceil((L_i + s_new) / 64) > bt_stride, a page to be written (a sequence's
+ * partly filled last page, or a popped page) lies outside [0, num_blocks), or
+ * *free_count is outside [0, free_capacity], it writes MLA_ERR_DEVICE_CHECK to
+ * device_status; if the stack holds fewer pages than needed, it writes
+ * MLA_ERR_NO_FREE_PAGES.  Either way no length and no free count changes, and
+ * no token a reader can see changes (rows may have been copied into free pages
+ * or past a sequence's length, and block-table entries past its pages).
+ * Host checks (nulls, sizes, alignment) return MLA_ERR_INVALID_ARG.  The
+ * caller keeps the state consistent: a page in a block table must not also be
+ * on the free stack.  Two launches (a grid that copies rows, one CTA that
+ * checks and commits); no host synchronisation.
+ */
+int mla_append_latent(const void* rows, int s_new, void* kcache, int64_t num_blocks,
+                      int32_t* block_table, int bt_stride, int32_t* cache_seqlens, int batch,
+                      int32_t* free_pages, int free_capacity, int32_t* free_count,
+                      int32_t* device_status, void* stream);
+
+/*
+ * mla_release_pages -- give back the pages of finished sequences ("FlashMLA:
+ * Revolutionizing Efficient Decoding...", section 4.3.2: unused blocks are
+ * easily deallocated).
+ *
+ * For every i with release_mask[i] != 0 (batch order), pushes
+ * block_table[i][0 : ceil(L_i / 64)] onto the free stack in page order and sets
+ * cache_seqlens[i] = 0; *free_count grows by the pages pushed.  Block-table
+ * rows are not cleared (entries past a sequence's pages are never read).
+ * release_mask: device int32 [batch]; the other arguments as for
+ * mla_append_latent.  A negative length, ceil(L_i / 64) > bt_stride or a free
+ * count outside [0, free_capacity] writes MLA_ERR_DEVICE_CHECK, and pages that
+ * would overfill free_pages write MLA_ERR_NO_FREE_PAGES, to device_status; then
+ * nothing changes.  One CTA; no host synchronisation.
+ */
+int mla_release_pages(const int32_t* release_mask, int32_t* block_table, int bt_stride,
+                      int32_t* cache_seqlens, int batch, int32_t* free_pages, int free_capacity,
+                      int32_t* free_count, int32_t* device_status, void* stream);
 
 /* mla_error_string -- static text for a status code (never NULL). */
 const char* mla_error_string(int status);

@@ -26,10 +26,12 @@ MLA_ERR_CUDA = 3
 MLA_ERR_DEVICE_TIMEOUT = 4
 MLA_ERR_DEVICE_CHECK = 5
 MLA_ERR_SCRATCH_LIMIT = 6
+MLA_ERR_NO_FREE_PAGES = 7
 STATIC_SCRATCH_BYTES = 48 << 20
 
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-           "mla_decode_kvcache_static_scratch", "mla_error_string", "mla_version")
+           "mla_decode_kvcache_static_scratch", "mla_append_latent", "mla_release_pages",
+           "mla_error_string", "mla_version")
 
 
 class MLAError(RuntimeError):
@@ -59,6 +61,10 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache_static_scratch.argtypes = [p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
                                                       f32, i32, p, p, i32, p, p, p, p]
     lib.mla_decode_kvcache_static_scratch.restype = i32
+    lib.mla_append_latent.argtypes = [p, i32, p, i64, p, i32, p, i32, p, i32, p, p, p]
+    lib.mla_append_latent.restype = i32
+    lib.mla_release_pages.argtypes = [p, p, i32, p, i32, p, i32, p, p, p]
+    lib.mla_release_pages.restype = i32
     lib.mla_error_string.argtypes = [i32]
     lib.mla_error_string.restype = ctypes.c_char_p
     lib.mla_version.argtypes = []
@@ -153,3 +159,48 @@ def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch
             _ptr(out), _ptr(lse), _ptr(device_status), _stream_handle(dev))
         _check(rc, "mla_decode_kvcache")
     return out, lse
+
+
+def _check_state(block_table, cache_seqlens, free_pages, free_count, dev):
+    for t in (block_table, cache_seqlens, free_pages, free_count):
+        assert t.is_cuda and t.device == dev and t.is_contiguous() and t.dtype == torch.int32
+    assert block_table.dim() == 2 and block_table.shape[0] == cache_seqlens.numel()
+    assert free_count.numel() == 1
+
+
+def append_latent(rows: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
+                  cache_seqlens: torch.Tensor, free_pages: torch.Tensor, free_count: torch.Tensor,
+                  device_status: torch.Tensor | None = None):
+    """Append rows [b, s_new, 576] bf16 as the next s_new tokens of every sequence, taking
+    64-token pages off the free stack free_pages[:free_count].  Updates kcache, block_table,
+    cache_seqlens and free_count in place, on the current stream."""
+    b, s_new, d = rows.shape
+    dev = rows.device
+    assert rows.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
+    assert rows.is_contiguous() and kcache.is_contiguous() and kcache.device == dev
+    assert kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d == D_QK
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    assert cache_seqlens.numel() == b
+    with torch.cuda.device(dev):
+        _check(lib.mla_append_latent(_ptr(rows), s_new, _ptr(kcache), kcache.shape[0],
+                                     _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
+                                     b, _ptr(free_pages), free_pages.numel(), _ptr(free_count),
+                                     _ptr(device_status), _stream_handle(dev)),
+               "mla_append_latent")
+
+
+def release_pages(release_mask: torch.Tensor, block_table: torch.Tensor,
+                  cache_seqlens: torch.Tensor, free_pages: torch.Tensor, free_count: torch.Tensor,
+                  device_status: torch.Tensor | None = None):
+    """Push the pages of every sequence with release_mask[i] != 0 back onto the free stack and
+    set its length to 0 (in place, on the current stream)."""
+    dev = cache_seqlens.device
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    assert release_mask.dtype == torch.int32 and release_mask.device == dev
+    assert release_mask.is_contiguous() and release_mask.numel() == cache_seqlens.numel()
+    with torch.cuda.device(dev):
+        _check(lib.mla_release_pages(_ptr(release_mask), _ptr(block_table), block_table.shape[1],
+                                     _ptr(cache_seqlens), cache_seqlens.numel(), _ptr(free_pages),
+                                     free_pages.numel(), _ptr(free_count), _ptr(device_status),
+                                     _stream_handle(dev)),
+               "mla_release_pages")

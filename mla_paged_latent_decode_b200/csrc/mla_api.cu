@@ -152,6 +152,9 @@ const char* mla_error_string(int status) {
     case MLA_ERR_SCRATCH_LIMIT:
       return "MLA_ERR_SCRATCH_LIMIT: workspace needed exceeds the library's static scratch "
              "(MLA_STATIC_SCRATCH_BYTES)";
+    case MLA_ERR_NO_FREE_PAGES:
+      return "MLA_ERR_NO_FREE_PAGES: too few free pages for an append, or no room on the free "
+             "list for a release";
     default: return "unknown mla status";
   }
 }

@@ -46,7 +46,37 @@ struct CombineParams {
   int batch, s_q, h_q, rows;
 };
 
+// Append of new tokens' rows to the paged cache (mla_paged_cache.cu).
+struct AppendParams {
+  const uint4* rows;          // [batch, s_new, 576] bf16 as 72 16-byte vectors per row
+  uint4* kcache;              // [num_blocks * 64, 576] bf16, likewise
+  int32_t* block_table;       // [batch, bt_stride]
+  const int32_t* seqlens;     // [batch], read by both kernels
+  int32_t* seqlens_rw;        // the same array, written by the commit kernel only
+  const int32_t* free_pages;  // [free_capacity]
+  const int32_t* free_count;  // [1], read by both kernels
+  int32_t* free_count_rw;     // the same word, written by the commit kernel only
+  int32_t* status;            // nullable
+  int64_t num_blocks;
+  int64_t bt_stride;
+  int batch, s_new, free_capacity;
+  int seqs_per_cta, tokens_per_cta;  // set by launch_append
+};
+
+struct ReleaseParams {
+  const int32_t* release_mask;  // [batch], nonzero = release
+  const int32_t* block_table;   // [batch, bt_stride]
+  int32_t* seqlens;             // [batch]
+  int32_t* free_pages;          // [free_capacity]
+  int32_t* free_count;          // [1]
+  int32_t* status;              // nullable
+  int64_t bt_stride;
+  int batch, free_capacity;
+};
+
 // Launchers (return cudaGetLastError() of their launch).
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_release(const ReleaseParams& p, cudaStream_t stream);
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,
                             int32_t* tile_md, int32_t* num_splits, cudaStream_t stream);
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,

@@ -45,7 +45,7 @@ def test_library_links_no_cuda_driver_or_torch():
 
 
 def test_error_strings():
-    for code in range(6):
+    for code in range(8):
         assert binding.error_string(code).startswith("MLA_")
     assert "unknown" in binding.error_string(99)
     assert "sm_100a" in binding.version()
@@ -103,3 +103,39 @@ def test_metadata_host_validation():
     assert binding.lib.mla_get_metadata(v(4096), 2, 16, 1, v(4096), v(4096), 0, v(0)) == 1
     nw, st = ctypes.c_int(0), ctypes.c_int(0)
     assert binding.lib.mla_metadata_shape(0, 16, 1, ctypes.byref(nw), ctypes.byref(st)) == 1
+
+
+def _append_raw(**kw):
+    args = dict(rows=1 << 12, s_new=1, kcache=1 << 12, num_blocks=4, block_table=1 << 12,
+                bt_stride=3, seqlens=1 << 12, batch=2, free_pages=1 << 12, free_capacity=4,
+                free_count=1 << 12)
+    args.update(kw)
+    v = ctypes.c_void_p
+    return binding.lib.mla_append_latent(
+        v(args["rows"]), args["s_new"], v(args["kcache"]), args["num_blocks"],
+        v(args["block_table"]), args["bt_stride"], v(args["seqlens"]), args["batch"],
+        v(args["free_pages"]), args["free_capacity"], v(args["free_count"]), v(0), v(0))
+
+
+@pytest.mark.parametrize("kw", [dict(rows=0), dict(kcache=0), dict(block_table=0),
+                                dict(seqlens=0), dict(free_pages=0), dict(free_count=0),
+                                dict(s_new=0), dict(s_new=65537), dict(batch=0),
+                                dict(batch=65537), dict(bt_stride=0), dict(free_capacity=0),
+                                dict(num_blocks=0), dict(num_blocks=1 << 25),
+                                dict(rows=(1 << 12) + 8), dict(kcache=(1 << 12) + 4)])
+def test_append_host_validation(kw):
+    assert _append_raw(**kw) == binding.MLA_ERR_INVALID_ARG
+
+
+def test_release_host_validation():
+    v = ctypes.c_void_p
+    ok = dict(mask=1 << 12, bt=1 << 12, stride=3, sl=1 << 12, batch=2, fp=1 << 12, cap=4, fc=1 << 12)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return binding.lib.mla_release_pages(v(a["mask"]), v(a["bt"]), a["stride"], v(a["sl"]),
+                                             a["batch"], v(a["fp"]), a["cap"], v(a["fc"]), v(0),
+                                             v(0))
+    for kw in (dict(mask=0), dict(bt=0), dict(sl=0), dict(fp=0), dict(fc=0), dict(stride=0),
+               dict(batch=0), dict(cap=0)):
+        assert call(**kw) == binding.MLA_ERR_INVALID_ARG
