@@ -307,13 +307,19 @@ def run_cuda(args, rank, local, world):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(args.workload, seed=0)
-    nbytes, flops = synth.algorithmic_work(inp)
+    fp8 = args.kv == "fp8"
+    nbytes, flops = synth.algorithmic_work(inp, 580 if fp8 else 1152)
     q = inp.q.to(dev)
     kc = inp.kcache.to(dev)
     bt = inp.block_table.to(dev)
     sl = inp.cache_seqlens.to(dev)
     b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
     num_workers, _ = binding.metadata_shape(b, h_q, s_q)
+    kc8 = ks = None
+    if fp8:
+        kc8, ks = encode_cache_fp8(kc, dev)
+        del kc
+        kc = None
     out = torch.empty((b, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
     ws = torch.empty((binding.workspace_size(b, s_q, h_q, num_workers),), dtype=torch.uint8,
@@ -333,8 +339,12 @@ def run_cuda(args, rank, local, world):
         return binding.get_mla_metadata(sl, h_q, s_q, num_workers)
 
     def decode_call(md, ns):
-        binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal, out=out,
-                                   lse=lse, workspace=ws, device_status=status)
+        if fp8:
+            binding.mla_decode_kvcache_fp8(q, kc8, ks, bt, sl, 512, md, ns, inp.scale, inp.causal,
+                                           out=out, lse=lse, workspace=ws, device_status=status)
+        else:
+            binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal, out=out,
+                                       lse=lse, workspace=ws, device_status=status)
 
     def step():
         # nothing between the two calls: the decode kernel is a programmatic
@@ -435,8 +445,12 @@ def run_cuda(args, rank, local, world):
             dbt.copy_(hbt, non_blocking=True)
             dsl.copy_(hsl, non_blocking=True)
             md, ns = binding.get_mla_metadata(dsl, h_q, s_q, num_workers)
-            o, l = binding.mla_decode_kvcache(dq, kc, dbt, dsl, 512, md, ns, inp.scale,
-                                              inp.causal, out=out, lse=lse, workspace=ws)
+            if fp8:
+                o, l = binding.mla_decode_kvcache_fp8(dq, kc8, ks, dbt, dsl, 512, md, ns, inp.scale,
+                                                      inp.causal, out=out, lse=lse, workspace=ws)
+            else:
+                o, l = binding.mla_decode_kvcache(dq, kc, dbt, dsl, 512, md, ns, inp.scale,
+                                                  inp.causal, out=out, lse=lse, workspace=ws)
             hout.copy_(o, non_blocking=True)
             hlse.copy_(l, non_blocking=True)
 
@@ -464,7 +478,7 @@ def run_cuda(args, rank, local, world):
                "note": "q, block_table and cache_seqlens copied in, out and lse copied back each "
                        "step; the latent cache stays resident in HBM as in serving"}
 
-    append = None if args.no_append else measure_append(inp, dev, stream, flush_l2)
+    append = None if args.no_append else measure_append(inp, dev, stream, flush_l2, fp8=fp8)
 
     if rank != 0:
         return None
@@ -487,11 +501,15 @@ def run_cuda(args, rank, local, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q and latent cache, shuffled 64-token pages)",
         "config": workload_config(inp, {"parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                                        "num_workers": num_workers}),
+                                        "num_workers": num_workers,
+                                        "kv_cache": ("fp8: E4M3 codes + one power-of-two fp32 scale "
+                                                     "per token (580 B per token)") if fp8 else
+                                                    "bf16 (1152 B per token)"}),
         "tflops": tflops,
         "roofline_frac": max(t_hbm, t_tc) / (ms_per_step / 1e3),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                     "frac": achieved / peak,
+                     "traffic": None if fp8 else recorded_traffic(args.workload),
                      "kernel": "mla_decode_kvcache call (decode kernel + split combine)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s / 1.59 PFLOP/s"},
@@ -518,7 +536,33 @@ def run_cuda(args, rank, local, world):
     return line
 
 
-def measure_append(inp, dev, stream, flush_l2, calls=50):
+def encode_cache_fp8(kc, dev):
+    """The FP8 cache of a bf16 cache, written by the library's own quantising
+    append: every page is one 64-token "sequence" appended into an empty
+    block-table row, with the free stack ordered so that sequence p receives
+    page p."""
+    from mla_paged_latent_decode_b200 import binding
+    nblk = kc.shape[0]
+    kc8 = torch.empty((nblk, 64, 576), dtype=torch.uint8, device=dev)
+    ks = torch.empty((nblk, 64), dtype=torch.float32, device=dev)
+    bt = torch.zeros((nblk, 1), dtype=torch.int32, device=dev)
+    lens = torch.zeros((nblk,), dtype=torch.int32, device=dev)
+    free = torch.arange(nblk - 1, -1, -1, dtype=torch.int32, device=dev)
+    fc = torch.tensor([nblk], dtype=torch.int32, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    for p0 in range(0, nblk, 65536):  # at most 65536 sequences per call
+        n = min(65536, nblk - p0)
+        binding.append_latent_fp8(kc[p0:p0 + n], kc8, ks, bt[p0:p0 + n], lens[p0:p0 + n], free,
+                                  fc, status)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0 or int(fc.item()) != 0:
+        raise RuntimeError("building the FP8 cache failed")
+    if not torch.equal(bt[:, 0], torch.arange(nblk, dtype=torch.int32, device=dev)):
+        raise RuntimeError("FP8 cache pages out of order")
+    return kc8, ks
+
+
+def measure_append(inp, dev, stream, flush_l2, calls=50, fp8=False):
     """Time mla_append_latent (the latent-cache append with page allocation) on
     the workload's batch: every sequence sits at a page boundary, so every call
     takes one new page per sequence (the costliest decode step), for s_new = s_q
@@ -535,6 +579,8 @@ def measure_append(inp, dev, stream, flush_l2, calls=50):
         pool = b * (1 + new_pages)
         gen = torch.Generator().manual_seed(1)
         kc = torch.randn((pool, 64, 576), generator=gen).to(torch.bfloat16).to(dev)
+        kc8 = torch.zeros((pool, 64, 576), dtype=torch.uint8, device=dev) if fp8 else None
+        ks = torch.zeros((pool, 64), dtype=torch.float32, device=dev) if fp8 else None
         rows = torch.randn((b, s_new, 576), generator=gen).to(torch.bfloat16).to(dev)
         perm = torch.randperm(pool, generator=gen).to(torch.int32)
         bt0 = torch.zeros((b, 1 + new_pages), dtype=torch.int32)
@@ -552,7 +598,10 @@ def measure_append(inp, dev, stream, flush_l2, calls=50):
             fc.copy_(fc0)
 
         def call():
-            binding.append_latent(rows, kc, bt, sl, free, fc, status)
+            if fp8:
+                binding.append_latent_fp8(rows, kc8, ks, bt, sl, free, fc, status)
+            else:
+                binding.append_latent(rows, kc, bt, sl, free, fc, status)
 
         for _ in range(3):
             restore()
@@ -576,7 +625,7 @@ def measure_append(inp, dev, stream, flush_l2, calls=50):
         torch.cuda.synchronize(dev)
         del graph
         us = statistics.median(a.elapsed_time(z) for a, z in evs) * 1e3
-        nbytes = 2 * b * s_new * 1152 + 16 * b
+        nbytes = b * s_new * (1152 + (580 if fp8 else 1152)) + 16 * b
         res[name] = {"s_new": s_new, "batch": b, "us": us, "bytes": nbytes,
                      "gb_s": nbytes / (us * 1e-6) / 1e9, "launches": 2,
                      "note": "every sequence takes a new page; L2 flushed before each call"}
@@ -589,7 +638,11 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", default="dsv3_decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(synth.WORKLOADS),
+                    help="default: dsv3_decode (bf16 cache) or varlen_h16 (fp8 cache)")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="latent cache format (fp8: E4M3 codes + per-token scale; "
+                         "up to 64 query rows per sequence)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
     ap.add_argument("--no-append", action="store_true",
@@ -597,6 +650,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="approximate oracle time for the cpu_baseline sample")
     args = ap.parse_args()
+    if args.workload is None:
+        args.workload = "varlen_h16" if args.kv == "fp8" else "dsv3_decode"
     if args.warmup < 3 and args.impl == "cuda":
         raise SystemExit("--warmup must be at least 3")
     rank, local, world = dist_setup(args.gpus)

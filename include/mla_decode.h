@@ -239,6 +239,55 @@ int mla_append_latent(const void* rows, int s_new, void* kcache, int64_t num_blo
                       int32_t* device_status, void* stream);
 
 /*
+ * mla_append_latent_fp8 -- mla_append_latent for an FP8 latent cache: each new
+ * bf16 row is encoded into 576 E4M3 codes and one per-token scale as it is
+ * written.
+ *
+ * The pages name FP8 support as the next way to cut the cache's memory
+ * ("FlashMLA: Revolutionizing Efficient Decoding...", section 9 "Future
+ * Directions") and give no format.  The format here: E4M3 codes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, largest finite value 448) and a
+ * scale 2^k per token, k the smallest integer with max_c |x_c| <= 448 * 2^k
+ * (k = 0 for an all-zero row); code_c is x_c / 2^k rounded to the nearest E4M3
+ * value, ties to even, sign kept.  The decode uses code * 2^k, which is exact.
+ *
+ * kcache:  device uint8 [num_blocks, 64, 576] E4M3 codes, 16-byte aligned.
+ * kscale:  device fp32 [num_blocks, 64] scales, 16-byte aligned.
+ * Everything else (pages, block table, lengths, free stack, checks, status,
+ * launches) is as for mla_append_latent.
+ */
+int mla_append_latent_fp8(const void* rows, int s_new, void* kcache, float* kscale,
+                          int64_t num_blocks, int32_t* block_table, int bt_stride,
+                          int32_t* cache_seqlens, int batch, int32_t* free_pages,
+                          int free_capacity, int32_t* free_count, int32_t* device_status,
+                          void* stream);
+
+/*
+ * mla_decode_kvcache_fp8 -- the decode over an FP8 latent cache (written by
+ * mla_append_latent_fp8): the same operation as mla_decode_kvcache with each
+ * cached row K_t = code_t * scale_t.  The cache moves half the bytes of the
+ * bf16 cache; each page is widened to bf16 inside the decode kernel, exactly.
+ *
+ * kcache:  device uint8 [num_blocks, 64, 576] E4M3 codes, 16-byte aligned.
+ * kscale:  device fp32 [num_blocks, 64] per-token scales, 16-byte aligned.
+ * Rows of a sequence's last page past its length are never read as data (the
+ * kernel zeroes them), so their codes and scales may hold anything.  Widening
+ * is exact for scales 2^k with -124 <= k <= 67 (what the quantising append
+ * writes for rows whose largest magnitude lies in about [1e-35, 6.6e22]).
+ * Requires s_q * h_q <= 64 query rows per sequence (MLA_ERR_UNSUPPORTED
+ * otherwise); metadata from mla_get_metadata as for mla_decode_kvcache.  All
+ * other arguments, the workspace, errors and launches are as for
+ * mla_decode_kvcache.
+ */
+int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscale,
+                           int64_t num_blocks, const int32_t* block_table, int bt_stride,
+                           const int32_t* cache_seqlens, int batch, int s_q, int h_q, int d,
+                           int dv, float softmax_scale, int causal, const int32_t* tile_md,
+                           const int32_t* num_splits, int num_workers, void* workspace,
+                           size_t workspace_bytes, void* out, float* lse,
+                           int32_t* device_status, void* stream);
+
+/*
  * mla_release_pages -- give back the pages of finished sequences ("FlashMLA:
  * Revolutionizing Efficient Decoding...", section 4.3.2: unused blocks are
  * easily deallocated).

@@ -31,7 +31,7 @@ STATIC_SCRATCH_BYTES = 48 << 20
 
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
            "mla_decode_kvcache_static_scratch", "mla_append_latent", "mla_release_pages",
-           "mla_error_string", "mla_version")
+           "mla_append_latent_fp8", "mla_decode_kvcache_fp8", "mla_error_string", "mla_version")
 
 
 class MLAError(RuntimeError):
@@ -63,6 +63,11 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache_static_scratch.restype = i32
     lib.mla_append_latent.argtypes = [p, i32, p, i64, p, i32, p, i32, p, i32, p, p, p]
     lib.mla_append_latent.restype = i32
+    lib.mla_append_latent_fp8.argtypes = [p, i32, p, p, i64, p, i32, p, i32, p, i32, p, p, p]
+    lib.mla_append_latent_fp8.restype = i32
+    lib.mla_decode_kvcache_fp8.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, f32,
+                                           i32, p, p, i32, p, sz, p, p, p, p]
+    lib.mla_decode_kvcache_fp8.restype = i32
     lib.mla_release_pages.argtypes = [p, p, i32, p, i32, p, i32, p, p, p]
     lib.mla_release_pages.restype = i32
     lib.mla_error_string.argtypes = [i32]
@@ -204,3 +209,62 @@ def release_pages(release_mask: torch.Tensor, block_table: torch.Tensor,
                                      free_pages.numel(), _ptr(free_count), _ptr(device_status),
                                      _stream_handle(dev)),
                "mla_release_pages")
+
+
+def append_latent_fp8(rows: torch.Tensor, kcache8: torch.Tensor, kscale: torch.Tensor,
+                      block_table: torch.Tensor, cache_seqlens: torch.Tensor,
+                      free_pages: torch.Tensor, free_count: torch.Tensor,
+                      device_status: torch.Tensor | None = None):
+    """append_latent for an FP8 cache: rows [b, s_new, 576] bf16 are encoded into E4M3
+    codes (kcache8 [nblk, 64, 576] uint8) and per-token scales (kscale [nblk, 64] fp32)."""
+    b, s_new, d = rows.shape
+    dev = rows.device
+    assert rows.dtype == torch.bfloat16 and rows.is_contiguous() and d == D_QK
+    assert kcache8.dtype == torch.uint8 and kcache8.is_contiguous() and kcache8.device == dev
+    assert kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == D_QK
+    assert kscale.dtype == torch.float32 and kscale.is_contiguous()
+    assert tuple(kscale.shape) == tuple(kcache8.shape[:2])
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    assert cache_seqlens.numel() == b
+    with torch.cuda.device(dev):
+        _check(lib.mla_append_latent_fp8(_ptr(rows), s_new, _ptr(kcache8), _ptr(kscale),
+                                         kcache8.shape[0], _ptr(block_table), block_table.shape[1],
+                                         _ptr(cache_seqlens), b, _ptr(free_pages),
+                                         free_pages.numel(), _ptr(free_count),
+                                         _ptr(device_status), _stream_handle(dev)),
+               "mla_append_latent_fp8")
+
+
+def mla_decode_kvcache_fp8(q: torch.Tensor, kcache8: torch.Tensor, kscale: torch.Tensor,
+                           block_table: torch.Tensor, cache_seqlens: torch.Tensor, dv: int,
+                           tile_md: torch.Tensor, num_splits: torch.Tensor,
+                           softmax_scale: float, causal: bool = False,
+                           out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None,
+                           device_status: torch.Tensor | None = None):
+    """Paged MLA decode over an FP8 cache (codes kcache8 [nblk, 64, 576] uint8 and per-token
+    scales kscale [nblk, 64] fp32).  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q])."""
+    b, s_q, h_q, d = q.shape
+    dev = q.device
+    for t in (q, kcache8, kscale, block_table, cache_seqlens, tile_md, num_splits):
+        assert t.is_cuda and t.device == dev and t.is_contiguous()
+    assert q.dtype == torch.bfloat16 and kcache8.dtype == torch.uint8
+    assert kscale.dtype == torch.float32 and tuple(kscale.shape) == tuple(kcache8.shape[:2])
+    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
+    assert kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == d
+    num_workers = tile_md.shape[0]
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty((b, s_q, h_q, dv), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+        need = workspace_size(b, s_q, h_q, num_workers, dv)
+        if workspace is None:
+            workspace = torch.empty((max(need, 256),), dtype=torch.uint8, device=dev)
+        rc = lib.mla_decode_kvcache_fp8(
+            _ptr(q), _ptr(kcache8), _ptr(kscale), kcache8.shape[0], _ptr(block_table),
+            block_table.shape[1], _ptr(cache_seqlens), b, s_q, h_q, d, dv, float(softmax_scale),
+            int(bool(causal)), _ptr(tile_md), _ptr(num_splits), num_workers, _ptr(workspace),
+            workspace.numel(), _ptr(out), _ptr(lse), _ptr(device_status), _stream_handle(dev))
+        _check(rc, "mla_decode_kvcache_fp8")
+    return out, lse

@@ -113,6 +113,22 @@ bool make_chunk_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t 
   return r == CUDA_SUCCESS;
 }
 
+// The E4M3 cache viewed as 3-D {192 bytes, rows, 3 parts} (strides: a row is
+// 576 bytes, a part 192): one box of 192 x 64 x 3 brings a whole page, each part
+// landing as 64 rows x 192 bytes.  No swizzle; the converter warps read it.
+bool make_fp8_page_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {192, static_cast<cuuint64_t>(rows), 3};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk), 192};
+  cuuint32_t box[3] = {192, 64, 3};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Query rows up to 64 per sequence run on single CTAs (one 64-row block); more
@@ -136,6 +152,9 @@ int workers_for(int sms, int s_q, int h_q, int* out) {
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int launch_combine_for(const int32_t* num_splits, float* part_o, float* part_lse, void* out,
+                       float* lse, int batch, int s_q, int h_q, int rows, cudaStream_t st);
 
 }  // namespace
 
@@ -270,6 +289,75 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
     if (mla::launch_decode(tm_q, tm_page, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
   }
 
+  return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
+}
+
+int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscale,
+                           int64_t num_blocks, const int32_t* block_table, int bt_stride,
+                           const int32_t* cache_seqlens, int batch, int s_q, int h_q, int d,
+                           int dv, float softmax_scale, int causal, const int32_t* tile_md,
+                           const int32_t* num_splits, int num_workers, void* workspace,
+                           size_t workspace_bytes, void* out, float* lse,
+                           int32_t* device_status, void* stream) {
+  if (q == nullptr || kcache == nullptr || kscale == nullptr || block_table == nullptr ||
+      cache_seqlens == nullptr || tile_md == nullptr || num_splits == nullptr || out == nullptr ||
+      lse == nullptr || workspace == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (d != mla::kDqk || dv != mla::kDv) return MLA_ERR_UNSUPPORTED;
+  if (batch < 1 || s_q < 1 || h_q < 1 || bt_stride < 1 || num_workers < 1 ||
+      num_workers > (1 << 20) || (causal != 0 && causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (uses_pairs(s_q, h_q)) return MLA_ERR_UNSUPPORTED;  // more than 64 query rows
+  if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * s_q * h_q >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(kscale, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 256) || !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_workspace_size(batch, s_q, h_q, dv, num_workers);
+  if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
+
+  const int rows = s_q * h_q;
+  CUtensorMap tm_q, tm_page8;
+  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
+  if (!make_fp8_page_map(&tm_page8, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage))
+    return MLA_ERR_CUDA;
+  const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             round_up(slots * rows * dv * sizeof(float), 256));
+  mla::DecodeParams p{};
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.status = device_status;
+  p.kscale = kscale;
+  p.bt_stride = bt_stride;
+  p.num_blocks = num_blocks;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = rows;
+  p.causal = causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mla::launch_decode_fp8(tm_q, tm_page8, p, num_workers, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
+}
+
+}  // extern "C"
+
+namespace {
+// The split combine after either decode kernel (it has work only where a
+// sequence has more than one piece).
+int launch_combine_for(const int32_t* num_splits, float* part_o, float* part_lse, void* out,
+                       float* lse, int batch, int s_q, int h_q, int rows, cudaStream_t st) {
   mla::CombineParams c{};
   c.num_splits = num_splits;
   c.part_o = part_o;
@@ -283,5 +371,4 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   if (mla::launch_combine(c, st) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }
-
-}  // extern "C"
+}  // namespace

@@ -39,43 +39,56 @@
 // re-designed for the 5th-generation tensor core: operands and accumulators
 // live in tensor memory, MMAs are issued by one thread, and the softmax runs in
 // warps of its own.
+#include <cuda_bf16.h>
+
 #include "mla_kernels.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
 
-constexpr int kThreads = 256;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;    // issues QK^T of even pages; allocates tensor memory
 constexpr int kPvWarp = 6;     // issues PV
 constexpr int kQkOddWarp = 7;  // issues QK^T of odd pages
+constexpr int kConvWarp0 = 8;  // FP8 cache: first of four converter warps
+constexpr int kConvThreads = 128;
+constexpr int kConvBarrier = 1;                    // named barrier of the converter warps
 constexpr int kChunkBytes = 64 * 128;              // 64 rows x 64 bf16 (one swizzle column block)
 constexpr int kChunks = kDqk / 64;                 // 9
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 73728 = 64 x 576 bf16
-constexpr int kStages = 3;
 constexpr int kPBytes = 64 * 128;                  // P: 64 rows x 64 tokens bf16
+constexpr int kFp8PageBytes = kPage * kDqk;        // 36864: one page of E4M3 codes
+constexpr int kFp8PartBytes = 192;                 // a row's codes arrive as 3 parts of 192 bytes
+constexpr int kFp8SlotBytes = kFp8PageBytes + kPage * 4;  // codes + the page's 64 fp32 scales
 
-constexpr int kOffKV = 0;
-constexpr int kOffP = kOffKV + kStages * kTileBytes;
-constexpr int kOffBar = kOffP + kPBytes;
-enum Bar {
-  kFull0 = 0,
-  kEmpty0 = kStages,
-  kQFull = 2 * kStages,
-  kSFull0,
-  kSFull1,
-  kSFree0,
-  kSFree1,
-  kPFull,
-  kPvDone,
-  kOFull,
-  kNumBars
+// Shared-memory layout, barriers and threads of the bf16-cache kernel
+// (kFp8 = false) and of the FP8-cache kernel (kFp8 = true).  The FP8 kernel
+// stages each page's codes and scales in one of two slots; converter warps
+// widen them into the same bf16 tile layout the MMAs read, so its ring of
+// bf16 tiles has two stages instead of three.
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kThreads = kFp8 ? 256 + kConvThreads : 256;
+  static constexpr int kStages = kFp8 ? 2 : 3;
+  static constexpr int kSlots = kFp8 ? 2 : 0;
+  static constexpr int kOffKV = 0;
+  static constexpr int kOffP = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffSlot = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffSlot + kSlots * kFp8SlotBytes;
+  static constexpr int kFull0 = 0, kEmpty0 = kStages, kQFull = 2 * kStages;
+  static constexpr int kSFull0 = kQFull + 1, kSFull1 = kQFull + 2;
+  static constexpr int kSFree0 = kQFull + 3, kSFree1 = kQFull + 4;
+  static constexpr int kPFull = kQFull + 5, kPvDone = kQFull + 6, kOFull = kQFull + 7;
+  static constexpr int kSlotFull0 = kQFull + 8, kSlotEmpty0 = kSlotFull0 + kSlots;
+  static constexpr int kNumBars = kSlotEmpty0 + kSlots;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem address + abort flag
+  static constexpr int kSmemUsed = kOffMisc + 16;
+  static constexpr int kSmemBytes = kSmemUsed + 1024;      // slack to align the base to 1024 B
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kOffP % 1024 == 0 && kOffSlot % 16 == 0, "alignment");
 };
-constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem address + abort flag
-constexpr int kSmemUsed = kOffMisc + 16;
-constexpr int kSmemBytes = kSmemUsed + 1024;       // slack to align the base to 1024 B
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQ = 0;                     // lanes 0-15, columns 0..287
@@ -86,7 +99,6 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units: P <= 2^8 befor
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
 
-static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kTmemS + 128 <= kTmemCols, "tensor memory budget");
 
 struct Piece {
@@ -123,17 +135,44 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// E4M3 -> bf16 without the conversion unit (whose throughput is a small
+// fraction of the integer and FMA pipes').  For a code b = s eeee mmm, the
+// 16-bit pattern s 0000 eeee mmm 0000 is the bf16 value b * 2^-120 (E4M3
+// subnormals become bf16 subnormals, zero stays zero).  Two exact bf16x2
+// multiplies, by 2^60 and by 2^60 * scale, then give b * scale: every step is
+// exact for scales 2^k with -124 <= k <= 67 (below -124 the smallest codes
+// times the scale fall under bf16's range).
+//   bytes2: the two codes sit in bytes sel selects (0x1404: bytes 0, 1;
+//   0x3424: bytes 2, 3); lo code -> low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t word, uint32_t sel,
+                                                     uint32_t f_hi, uint32_t f_lo) {
+  const uint32_t t = __byte_perm(word, 0u, sel);  // (b_hi << 24) | (b_lo << 8)
+  const uint32_t pat = ((t & 0x7F007F00u) >> 4) | (t & 0x80008000u);
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pat);
+  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_hi));
+  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_lo));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_page, const DecodeParams p) {
+  using C = Cfg<kFp8>;
+  constexpr int kStages = C::kStages;
+  constexpr int kFull0 = C::kFull0, kEmpty0 = C::kEmpty0, kQFull = C::kQFull;
+  constexpr int kSFull0 = C::kSFull0, kSFull1 = C::kSFull1, kSFree0 = C::kSFree0;
+  constexpr int kSFree1 = C::kSFree1, kPFull = C::kPFull, kPvDone = C::kPvDone;
+  constexpr int kOFull = C::kOFull;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* skv = smem + kOffKV;
-  uint8_t* sp = smem + kOffP;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  uint8_t* skv = smem + C::kOffKV;
+  uint8_t* sp = smem + C::kOffP;
+  uint8_t* sslot = smem + C::kOffSlot;  // FP8 cache only
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   // Launched as a programmatic dependent of the scheduler kernel: its CTAs may
   // start while the scheduler runs, and read the metadata only after this wait.
@@ -161,6 +200,10 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar[kPFull], kSoftmaxThreads);
     mbar_init(&bar[kPvDone], 1);
     mbar_init(&bar[kOFull], 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&bar[C::kSlotFull0 + s], 1);
+      mbar_init(&bar[C::kSlotEmpty0 + s], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -172,10 +215,135 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // FP8 cache: 384 threads launched with 168 registers each; the softmax
+  // warpgroup raises its budget to 232, the single-thread roles (warps 4-7)
+  // lower theirs to 56 and the converters to 96: 49152 of the 64512 in all.
+  constexpr int kNSlots = kFp8 ? C::kSlots : 1;  // keeps the bf16 instantiation well formed
+  if constexpr (kFp8) {
+    if (warp >= 4 && warp < kConvWarp0) setmaxnreg_dec<56>();
+  }
 
   // The stage ring carries, per piece with pages, one entry for the query rows
   // followed by one entry per page; every role counts entries the same way.
-  if (warp == kTmaWarp) {
+  if (kFp8 && warp == kTmaWarp) {
+    // ------------------------------------------------------------ FP8 page producer
+    // Each page's codes (one 3-D box: 3 parts x 64 rows x 192 bytes) and its 64
+    // scales go to the next staging slot; the converter warps take it from there.
+    if (lane == 0) {
+      prefetch_tensormap(&tm_page);
+      int g = 0;
+      bool ok = true;
+      for (int pc = 0; pc < npieces && ok; ++pc) {
+        const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+        if (p.seqlens[pz.seq] > p.bt_stride * kPage) report(p.status, MLA_ERR_DEVICE_CHECK);
+        const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+        for (int e = 0; e < pz.npg; ++e, ++g) {
+          const int slot = g % kNSlots, use = g / kNSlots;
+          if (use > 0) {
+            ok = mbar_wait(&bar[C::kSlotEmpty0 + slot], (use - 1) & 1, abort_flag, kWaitLimitNs);
+            if (!ok) break;
+          }
+          uint8_t* dst = sslot + slot * kFp8SlotBytes;
+          int page = __ldg(bt + pz.pg0 + e);
+          // The tensor map bounds the codes load, but the untiled scale copy has
+          // no bounds: a page id outside the cache is reported and replaced.
+          if (page < 0 || page >= p.num_blocks) {
+            report(p.status, MLA_ERR_DEVICE_CHECK);
+            page = 0;
+          }
+          mbar_arrive_expect_tx(&bar[C::kSlotFull0 + slot], kFp8SlotBytes);
+          tma_load_3d(dst, &tm_page, 0, page * kPage, 0, &bar[C::kSlotFull0 + slot]);
+          bulk_load(dst + kFp8PageBytes, p.kscale + static_cast<int64_t>(page) * kPage, kPage * 4,
+                    &bar[C::kSlotFull0 + slot]);
+        }
+      }
+      for (int s = 0; s < kNSlots && s < g; ++s) {  // let every copy land (bounded)
+        const int n = g - 1 - s;
+        mbar_wait(&bar[C::kSlotFull0 + n % kNSlots], (n / kNSlots) & 1, abort_flag,
+                  kWaitLimitNs);
+      }
+    }
+  } else if (kFp8 && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ FP8 converters
+    // Producers of the bf16 ring: the query rows of a piece by TMA (thread 0),
+    // and each page widened from its staging slot into the swizzled bf16 tile
+    // (row r, dims 16i..16i+15 per item).  Rows past the sequence's end are
+    // written as zeros, so stale codes or scales there never reach an MMA.
+    // The four warps decide together after a named barrier, so that a wait
+    // that gave up in one warp stops all of them at the same point.
+    if constexpr (kFp8) setmaxnreg_dec<96>();
+    const int ct = threadIdx.x - kConvWarp0 * 32;
+    int entries = 0, g = 0;
+    for (int pc = 0; pc < npieces; ++pc) {
+      const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+      if (pz.npg == 0) continue;
+      const int L = p.seqlens[pz.seq];
+      bool stop = false;
+      for (int e = -1; e < pz.npg; ++e) {
+        const int stage = entries % kStages, use = entries / kStages;
+        if (use > 0) warp_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag);
+        uint8_t* dst = skv + stage * kTileBytes;
+        if (e < 0) {
+          named_bar_sync(kConvBarrier, kConvThreads);
+          if (*abort_flag) { stop = true; break; }
+          if (ct == 0) {
+            const int qrow = pz.seq * p.rows + blockIdx.y * kRowsPerCta;
+            mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
+          }
+        } else {
+          const int slot = g % kNSlots;
+          if (!*abort_flag)
+            warp_wait(&bar[C::kSlotFull0 + slot], (g / kNSlots) & 1, abort_flag);
+          named_bar_sync(kConvBarrier, kConvThreads);
+          if (*abort_flag) { stop = true; break; }
+          const uint8_t* src = sslot + slot * kFp8SlotBytes;
+          const float* scales = reinterpret_cast<const float*>(src + kFp8PageBytes);
+          const int valid = L - (pz.pg0 + e) * kPage;  // rows of this page inside the sequence
+          for (int it = ct; it < kPage * (kDqk / 16); it += kConvThreads) {
+            const int r = it / (kDqk / 16), i = it - r * (kDqk / 16);
+            uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+            if (r < valid) {
+              const uint4 v = *reinterpret_cast<const uint4*>(
+                  src + (i / 12) * (kPage * kFp8PartBytes) + r * kFp8PartBytes + (i % 12) * 16);
+              // 2^60 * scale as bf16x2 (a power of two: its fp32 bits end in 16 zeros)
+              const uint32_t f_lo = (__float_as_uint(scales[r] * 0x1p60f) >> 16) * 0x10001u;
+              constexpr uint32_t f_hi = 0x5D805D80u;  // 2^60 in both halves
+              lo.x = e4m3x2_to_bf16x2(v.x, 0x1404u, f_hi, f_lo);
+              lo.y = e4m3x2_to_bf16x2(v.x, 0x3424u, f_hi, f_lo);
+              lo.z = e4m3x2_to_bf16x2(v.y, 0x1404u, f_hi, f_lo);
+              lo.w = e4m3x2_to_bf16x2(v.y, 0x3424u, f_hi, f_lo);
+              hi.x = e4m3x2_to_bf16x2(v.z, 0x1404u, f_hi, f_lo);
+              hi.y = e4m3x2_to_bf16x2(v.z, 0x3424u, f_hi, f_lo);
+              hi.z = e4m3x2_to_bf16x2(v.w, 0x1404u, f_hi, f_lo);
+              hi.w = e4m3x2_to_bf16x2(v.w, 0x3424u, f_hi, f_lo);
+            }
+            // dims 16i..16i+15: chunk i/4, 16-byte units 2(i%4) and 2(i%4)+1, swizzled by row
+            uint8_t* rowp = dst + (i >> 2) * kChunkBytes + r * 128;
+            const int u = 2 * (i & 3);
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (r & 7)) << 4)) = hi;
+          }
+          fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+          named_bar_sync(kConvBarrier, kConvThreads);
+          if (ct == 0) {
+            mbar_arrive(&bar[C::kSlotEmpty0 + slot]);
+            mbar_arrive(&bar[kFull0 + stage]);
+          }
+          ++g;
+        }
+        ++entries;
+      }
+      if (stop) break;
+    }
+    if (ct == 0) {  // let the query copies land before leaving (bounded)
+      for (int s = 0; s < kStages && s < entries; ++s) {
+        const int n = entries - 1 - s;
+        mbar_wait(&bar[kFull0 + n % kStages], (n / kStages) & 1, abort_flag, kWaitLimitNs);
+      }
+    }
+  } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
@@ -301,6 +469,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
+    if constexpr (kFp8) setmaxnreg_inc<232>();
     // 16-lane TMEM accesses: thread t holds rows t/4 and t/4 + 8 of its quarter's
     // 16, at columns 2(t%4) + {0,1} + 8g.
     const uint32_t quarter = static_cast<uint32_t>(32 * warp) << 16;
@@ -523,23 +692,52 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(mla_decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
+    e = cudaFuncSetAttribute(mla_decode_sm100_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_workers, row_blocks);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(Cfg<false>::kThreads);
+  cfg.dynamicSmemBytes = Cfg<false>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel, tm_q, tm_page, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel<false>, tm_q, tm_page, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
+                              const DecodeParams& p, int num_workers, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(mla_decode_sm100_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<true>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_workers, row_blocks);
+  cfg.blockDim = dim3(Cfg<true>::kThreads);
+  cfg.dynamicSmemBytes = Cfg<true>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel<true>, tm_q, tm_page8, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

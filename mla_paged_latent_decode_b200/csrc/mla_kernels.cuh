@@ -30,6 +30,7 @@ struct DecodeParams {
   float* part_o;        // [pieces, rows, 512]
   float* part_lse;      // [pieces, rows]
   int32_t* status;      // nullable
+  const float* kscale;  // FP8 cache only: [num_blocks * 64] per-token scales
   int64_t bt_stride;
   int64_t num_blocks;
   int batch, s_q, h_q, rows;  // rows = s_q * h_q
@@ -49,7 +50,9 @@ struct CombineParams {
 // Append of new tokens' rows to the paged cache (mla_paged_cache.cu).
 struct AppendParams {
   const uint4* rows;          // [batch, s_new, 576] bf16 as 72 16-byte vectors per row
-  uint4* kcache;              // [num_blocks * 64, 576] bf16, likewise
+  uint4* kcache;              // [num_blocks * 64, 576] bf16, likewise (bf16 cache)
+  uint8_t* kcache8;           // [num_blocks * 64, 576] E4M3 codes (FP8 cache)
+  float* kscale;              // [num_blocks * 64] per-token scales (FP8 cache)
   int32_t* block_table;       // [batch, bt_stride]
   const int32_t* seqlens;     // [batch], read by both kernels
   int32_t* seqlens_rw;        // the same array, written by the commit kernel only
@@ -75,13 +78,17 @@ struct ReleaseParams {
 };
 
 // Launchers (return cudaGetLastError() of their launch).
-cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, bool fp8, cudaStream_t stream);
 cudaError_t launch_release(const ReleaseParams& p, cudaStream_t stream);
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,
                             int32_t* tile_md, int32_t* num_splits, cudaStream_t stream);
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+// FP8 (E4M3) cache, up to 64 query rows per sequence: tm_page8 is the codes viewed
+// as {192 bytes, rows, 3 parts} with a box of 192 x 64 x 3.
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
+                              const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
                                const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,

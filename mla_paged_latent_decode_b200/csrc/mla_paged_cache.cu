@@ -19,13 +19,18 @@
 //      writes the new block-table entries.  It reads the lengths and the free
 //      count but writes neither; every write stays inside the buffers (a row or
 //      entry whose page is out of range is skipped).
-//   2. mla_append_commit_kernel (one CTA): checks the whole request, then grows
-//      every length by s_new and lowers the free count, or, if the request is
-//      invalid, reports the reason and changes neither.  Rows written by kernel
-//      1 for a failed request lie in free pages or past a sequence's length,
-//      and block-table entries past its pages: no reader sees them.
+//   2. mla_append_commit_kernel (one CTA, a programmatic dependent of 1): checks
+//      the whole request while kernel 1 copies, waits for kernel 1 to finish,
+//      then grows every length by s_new and lowers the free count, or, if the
+//      request is invalid, reports the reason and changes neither.  Rows that
+//      kernel 1 wrote for a refused request lie in free pages or past a
+//      sequence's length, and block-table entries past its pages: no reader
+//      sees them.
 // A release is one CTA: check, push, then zero the lengths and raise the count.
+#include <cuda_fp8.h>
+
 #include "mla_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -33,8 +38,9 @@ namespace {
 constexpr int kVecsPerRow = kDqk * 2 / 16;  // 72 16-byte vectors per cached row
 constexpr int kAppendThreads = 256;
 constexpr int kMaxSeqsPerCta = 128;
-constexpr int kMaxTokensPerCta = 8;
+constexpr int kMaxTokensPerCta = 32;
 constexpr int kMaxRowsPerCta = kMaxSeqsPerCta * kMaxTokensPerCta;
+constexpr int kCopyUnroll = 4;  // 16-byte loads in flight per thread
 constexpr int kCommitThreads = 1024;
 
 __device__ __forceinline__ int64_t pages_of(int64_t tokens) { return (tokens + kPage - 1) / kPage; }
@@ -70,30 +76,84 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// One row's E4M3 encoding, by one warp: lanes 0-23 hold 24 dims each.  The
+// scale is the smallest 2^k with max|x| <= 448 * 2^k (k from the exponent of
+// max|x|: max|x| = f * 2^e with f in [0.5, 1), k = e - 9 if f <= 0.875, else
+// e - 8), and each code is x / 2^k rounded to nearest even, sign kept.
+__device__ __forceinline__ void encode_row_e4m3(const uint4* src, uint8_t* dst_codes,
+                                                float* dst_scale, int lane) {
+  float x[24];
+  float amax = 0.f;
+  if (lane < 24) {
+#pragma unroll
+    for (int v = 0; v < 3; ++v) {
+      const uint4 w = __ldg(src + 3 * lane + v);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        x[8 * v + 2 * h] = __uint_as_float(ws[h] << 16);
+        x[8 * v + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 24; ++c) amax = fmaxf(amax, fabsf(x[c]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int k = 0;
+  if (amax > 0.f) {
+    int e = 0;
+    const float f = frexpf(amax, &e);
+    k = f <= 0.875f ? e - 9 : e - 8;
+  }
+  if (lane < 24) {
+    uint32_t packed[6];
+#pragma unroll
+    for (int q = 0; q < 6; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 pair = make_float2(ldexpf(x[4 * q + 2 * h], -k), ldexpf(x[4 * q + 2 * h + 1], -k));
+        const uint32_t two = __nv_cvt_float2_to_fp8x2(pair, __NV_SATFINITE, __NV_E4M3);
+        word |= (two & 0xFFFFu) << (16 * h);
+      }
+      packed[q] = word;
+    }
+    uint2* out = reinterpret_cast<uint2*>(dst_codes + 24 * lane);
+    out[0] = make_uint2(packed[0], packed[1]);
+    out[1] = make_uint2(packed[2], packed[3]);
+    out[2] = make_uint2(packed[4], packed[5]);
+  }
+  if (lane == 0) *dst_scale = ldexpf(1.f, k);
+}
+
+template <bool kFp8>
 __global__ void __launch_bounds__(kAppendThreads)
 mla_append_rows_kernel(AppendParams p) {
   __shared__ int64_t warp_vals[32];
   __shared__ int32_t seq_len[kMaxSeqsPerCta];
   __shared__ int64_t seq_off[kMaxSeqsPerCta];
-  __shared__ int64_t dst_row[kMaxRowsPerCta];
+  __shared__ int32_t dst_row[kMaxRowsPerCta];
+  // The commit kernel is a programmatic dependent: it may start checking now,
+  // and writes only after this grid has finished.
+  grid_launch_dependents();
   const int tid = threadIdx.x;
   const int s0 = blockIdx.x * p.seqs_per_cta;
   const int s1 = min(p.batch, s0 + p.seqs_per_cta);
   const int ns = s1 - s0;
-
-  // pages popped for the sequences before this CTA's first one
-  int64_t part = 0;
-  for (int i = tid; i < s0; i += blockDim.x) part += new_pages(p.seqlens[i], p.s_new);
-  const int64_t before = block_reduce(part, warp_vals, Sum());
   const int64_t fc = *p.free_count;
   const bool fc_ok = fc >= 0 && fc <= p.free_capacity;
+
+  // this CTA's lengths, and the pages popped for the sequences before them
+  for (int j = tid; j < ns; j += blockDim.x) seq_len[j] = p.seqlens[s0 + j];
+  int64_t part = 0;
+  for (int i = tid; i < s0; i += blockDim.x) part += new_pages(p.seqlens[i], p.s_new);
+  const int64_t before = block_reduce(part, warp_vals, Sum());  // also publishes seq_len
   if (tid == 0) {
     int64_t off = before;
     for (int j = 0; j < ns; ++j) {
-      const int32_t L = p.seqlens[s0 + j];
-      seq_len[j] = L;
       seq_off[j] = off;
-      off += new_pages(L, p.s_new);
+      off += new_pages(seq_len[j], p.s_new);
     }
   }
   __syncthreads();
@@ -124,7 +184,7 @@ mla_append_rows_kernel(AppendParams p) {
     for (int r = tid; r < nrows; r += blockDim.x) {
       const int j = r / nt;
       const int32_t L = seq_len[j];
-      int64_t dst = -1;
+      int32_t dst = -1;
       if (L >= 0) {
         const int64_t t = static_cast<int64_t>(L) + k0 + r % nt;
         const int64_t lp = t / kPage, first = pages_of(L);
@@ -137,17 +197,47 @@ mla_append_rows_kernel(AppendParams p) {
             if (slot >= 0) page = p.free_pages[slot];
           }
         }
-        if (page >= 0 && page < p.num_blocks) dst = page * kPage + t % kPage;
+        // num_blocks * 64 < 2^31 (checked on the host), so the row index fits
+        if (page >= 0 && page < p.num_blocks) dst = static_cast<int32_t>(page * kPage + t % kPage);
       }
       dst_row[r] = dst;
     }
     __syncthreads();
-    for (int v = tid; v < nrows * kVecsPerRow; v += blockDim.x) {
-      const int r = v / kVecsPerRow, c = v - r * kVecsPerRow;
-      const int64_t dst = dst_row[r];
-      if (dst < 0) continue;
-      const int64_t src = (static_cast<int64_t>(s0 + r / nt) * p.s_new + k0 + r % nt);
-      p.kcache[dst * kVecsPerRow + c] = __ldg(p.rows + src * kVecsPerRow + c);
+    if constexpr (kFp8) {
+      // one warp per row: encode into codes and a per-token scale
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int r = warp; r < nrows; r += blockDim.x >> 5) {
+        const int32_t dst = dst_row[r];
+        if (dst < 0) continue;
+        const int64_t src = static_cast<int64_t>(s0 + r / nt) * p.s_new + k0 + r % nt;
+        encode_row_e4m3(p.rows + src * kVecsPerRow, p.kcache8 + static_cast<int64_t>(dst) * kDqk,
+                        p.kscale + dst, lane);
+      }
+      __syncthreads();
+      continue;
+    }
+    // kCopyUnroll loads in flight per thread before their stores
+    const int nvec = nrows * kVecsPerRow;
+    for (int v0 = tid; v0 < nvec; v0 += blockDim.x * kCopyUnroll) {
+      uint4 buf[kCopyUnroll];
+      int64_t to[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int v = v0 + u * static_cast<int>(blockDim.x);
+        to[u] = -1;
+        if (v < nvec) {
+          const int r = v / kVecsPerRow, c = v - r * kVecsPerRow;
+          const int32_t dst = dst_row[r];
+          if (dst >= 0) {
+            const int64_t src = static_cast<int64_t>(s0 + r / nt) * p.s_new + k0 + r % nt;
+            buf[u] = __ldg(p.rows + src * kVecsPerRow + c);
+            to[u] = static_cast<int64_t>(dst) * kVecsPerRow + c;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u)
+        if (to[u] >= 0) p.kcache[to[u]] = buf[u];
     }
     __syncthreads();
   }
@@ -188,6 +278,9 @@ mla_append_commit_kernel(AppendParams p) {
   const int64_t fc = *p.free_count;
   int64_t total = 0;
   const int rc = check_append(p, fc, &total, warp_vals);
+  // The rows kernel reads the lengths and the free count: write them only once
+  // it has finished (this kernel is its programmatic dependent).
+  grid_dependency_wait();
   if (rc != MLA_OK) {
     if (threadIdx.x == 0) report(p.status, rc);
     return;
@@ -254,7 +347,7 @@ mla_release_kernel(ReleaseParams p) {
 
 }  // namespace
 
-cudaError_t launch_append(const AppendParams& p_in, cudaStream_t stream) {
+cudaError_t launch_append(const AppendParams& p_in, bool fp8, cudaStream_t stream) {
   AppendParams p = p_in;
   p.tokens_per_cta = p.s_new < kMaxTokensPerCta ? p.s_new : kMaxTokensPerCta;
   int spc = (kMaxTokensPerCta + p.tokens_per_cta - 1) / p.tokens_per_cta;
@@ -266,10 +359,24 @@ cudaError_t launch_append(const AppendParams& p_in, cudaStream_t stream) {
   int gy = 2048 / gx;
   if (gy < 1) gy = 1;
   if (gy > chunks) gy = chunks;
-  mla_append_rows_kernel<<<dim3(gx, gy), kAppendThreads, 0, stream>>>(p);
+  if (fp8)
+    mla_append_rows_kernel<true><<<dim3(gx, gy), kAppendThreads, 0, stream>>>(p);
+  else
+    mla_append_rows_kernel<false><<<dim3(gx, gy), kAppendThreads, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  mla_append_commit_kernel<<<1, kCommitThreads, 0, stream>>>(p);
+  // the commit kernel checks the request while the rows kernel copies
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kCommitThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, mla_append_commit_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -313,8 +420,43 @@ int mla_append_latent(const void* rows, int s_new, void* kcache, int64_t num_blo
   p.batch = batch;
   p.s_new = s_new;
   p.free_capacity = free_capacity;
-  return mla::launch_append(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MLA_OK
-                                                                                 : MLA_ERR_CUDA;
+  return mla::launch_append(p, false, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+int mla_append_latent_fp8(const void* rows, int s_new, void* kcache, float* kscale,
+                          int64_t num_blocks, int32_t* block_table, int bt_stride,
+                          int32_t* cache_seqlens, int batch, int32_t* free_pages,
+                          int free_capacity, int32_t* free_count, int32_t* device_status,
+                          void* stream) {
+  if (rows == nullptr || kcache == nullptr || kscale == nullptr || block_table == nullptr ||
+      cache_seqlens == nullptr || free_pages == nullptr || free_count == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (s_new < 1 || s_new > 65536 || batch < 1 || batch > 65536 || bt_stride < 1 ||
+      free_capacity < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(rows) || !aligned16(kcache) || !aligned16(kscale)) return MLA_ERR_INVALID_ARG;
+  mla::AppendParams p{};
+  p.rows = static_cast<const uint4*>(rows);
+  p.kcache8 = static_cast<uint8_t*>(kcache);
+  p.kscale = kscale;
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.seqlens_rw = cache_seqlens;
+  p.free_pages = free_pages;
+  p.free_count = free_count;
+  p.free_count_rw = free_count;
+  p.status = device_status;
+  p.num_blocks = num_blocks;
+  p.bt_stride = bt_stride;
+  p.batch = batch;
+  p.s_new = s_new;
+  p.free_capacity = free_capacity;
+  return mla::launch_append(p, true, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 int mla_release_pages(const int32_t* release_mask, int32_t* block_table, int bt_stride,

@@ -162,10 +162,12 @@ def custom_workload(batch: int, s_q: int, h_q: int, seqlens, causal: bool = Fals
                     causal=causal, pool_pages=pool_pages, scale=scale)
 
 
-def algorithmic_work(inp: DecodeInputs) -> tuple[int, int]:
+def algorithmic_work(inp: DecodeInputs, kv_bytes_per_token: int = D_QK * 2) -> tuple[int, int]:
     """(bytes, flops) the method must move or compute for one call.
 
-    bytes: every visible-or-not cached row once (576 bf16, read once because
+    kv_bytes_per_token: bytes of one cached row (1152 for bf16; 580 for 576
+    E4M3 codes plus a 4-byte scale).
+    bytes: every visible-or-not cached row once (576 values, read once because
     the value is the first 512 dims of the same row), q in, out and lse out,
     seqlens and the used block-table entries.
     flops: 2 * (576 + 512) per (query row, visible key) pair.
@@ -174,7 +176,7 @@ def algorithmic_work(inp: DecodeInputs) -> tuple[int, int]:
     lens = inp.cache_seqlens.tolist()
     total_tokens = sum(lens)
     n_pages = sum(pages_for(v) for v in lens)
-    nbytes = (total_tokens * D_QK * 2 + b * s_q * h_q * (D_QK * 2 + D_V * 2)
+    nbytes = (total_tokens * kv_bytes_per_token + b * s_q * h_q * (D_QK * 2 + D_V * 2)
               + b * h_q * s_q * 4 + 4 * (b + n_pages))
     pairs = 0
     for L in lens:

@@ -19,7 +19,7 @@ HEADER = os.path.join(ROOT, "include", "mla_decode.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
     out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\sT\s(mla_[a-z_]+)$", out, flags=re.M))
+    exported = set(re.findall(r"\sT\s(mla_[a-z0-9_]+)$", out, flags=re.M))
     assert set(declared_functions()) <= exported
 
 

@@ -116,7 +116,7 @@ def test_pins_reject_mutation(name, tmp_path):
     import importlib.util
     old, new = MUTATIONS[name]
     src = open(f8.__file__).read()
-    assert src.count(old) == 1, old
+    assert src.count(old) >= 1, old
     path = tmp_path / f"mut_{name}.py"
     path.write_text(src.replace(old, new))
     spec = importlib.util.spec_from_file_location(f"mut_{name}", path)
@@ -129,7 +129,7 @@ def test_pins_reject_mutation(name, tmp_path):
         try:
             for t in (test_known_codes, test_every_finite_code_round_trips,
                       test_rounding_matches_brute_force, test_ties_go_to_even_codes,
-                      test_encoding_error_is_half_a_step):
+                      test_encoding_error_is_half_a_step, test_grid_rounding_equals_table_rounding):
                 t()
             for a in (0.75, 224.5, 1e4):
                 test_scale_exponent_is_the_smallest_fitting_power(a)
@@ -138,3 +138,37 @@ def test_pins_reject_mutation(name, tmp_path):
     except (AssertionError, ValueError):
         failed = True
     assert failed, f"mutation {name} went undetected"
+
+
+def test_block_encoder_equals_row_encoder():
+    g = torch.Generator().manual_seed(5)
+    rows = (torch.randn((50, 576), generator=g) * torch.logspace(-5, 5, 50)[:, None]).to(
+        torch.bfloat16).double().numpy()
+    codes, scales = f8.encode_rows(rows, chunk=7)
+    for n in range(50):
+        c, s = f8.encode_row(rows[n])
+        np.testing.assert_array_equal(codes[n], c)
+        assert scales[n] == s
+
+
+def test_block_scale_rule_equals_scalar_rule():
+    amax = np.concatenate([[0.0, 448.0, 392.0, 392.0001, 224.0, 1.0, 0.875, 0.8750001],
+                           np.ldexp(np.random.default_rng(1).random(2000) + 0.5,
+                                    np.random.default_rng(2).integers(-140, 120, 2000))])
+    rows = np.zeros((amax.size, 576))
+    rows[:, 7] = amax
+    _, scales = f8.encode_rows(rows, chunk=333)
+    for a, s in zip(amax, scales):
+        assert s == 2.0 ** f8.scale_exponent(a), a
+
+
+def test_grid_rounding_equals_table_rounding():
+    g = np.random.default_rng(4)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)])
+    vals = f8.decode_codes(codes)
+    lo, hi = f8.decode_codes(np.arange(0, 0x7E)), f8.decode_codes(np.arange(1, 0x7F))
+    mids = (lo + hi) / 2
+    rand = np.ldexp(g.random(200000) + 0.5, g.integers(-14, 9, 200000))
+    rand = rand[rand <= 448] * np.where(g.random(rand.size) < 0.5, -1, 1)
+    for y in (vals, mids, -mids, rand, np.array([0.0, -0.0, 2.0 ** -12, -2.0 ** -12])):
+        np.testing.assert_array_equal(f8.e4m3_round_grid(y), f8.e4m3_round(y))
