@@ -113,17 +113,18 @@ bool make_chunk_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t 
   return r == CUDA_SUCCESS;
 }
 
-// The E4M3 cache viewed as 3-D {192 bytes, rows, 3 parts} (strides: a row is
-// 576 bytes, a part 192): one box of 192 x 64 x 3 brings a whole page, each part
-// landing as 64 rows x 192 bytes.  No swizzle; the converter warps read it.
+// The E4M3 cache as [rows, 576] bytes read in boxes of 128 bytes x 64 rows, no
+// swizzle.  The decode starts the box for chunk c at x = 64 c - 64, so that
+// chunk c lands in the upper 64 bytes of each 128-byte row slot (x < 0 is out
+// of bounds and filled with zeros).
 bool make_fp8_page_map(CUtensorMap* map, const void* base, uint64_t rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {192, static_cast<cuuint64_t>(rows), 3};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk), 192};
-  cuuint32_t box[3] = {192, 64, 3};
-  cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kDqk)};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

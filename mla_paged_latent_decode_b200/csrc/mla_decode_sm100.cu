@@ -59,35 +59,32 @@ constexpr int kChunkBytes = 64 * 128;              // 64 rows x 64 bf16 (one swi
 constexpr int kChunks = kDqk / 64;                 // 9
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 73728 = 64 x 576 bf16
 constexpr int kPBytes = 64 * 128;                  // P: 64 rows x 64 tokens bf16
-constexpr int kFp8PageBytes = kPage * kDqk;        // 36864: one page of E4M3 codes
-constexpr int kFp8PartBytes = 192;                 // a row's codes arrive as 3 parts of 192 bytes
-constexpr int kFp8SlotBytes = kFp8PageBytes + kPage * 4;  // codes + the page's 64 fp32 scales
 
 // Shared-memory layout, barriers and threads of the bf16-cache kernel
 // (kFp8 = false) and of the FP8-cache kernel (kFp8 = true).  The FP8 kernel
-// stages each page's codes and scales in one of two slots; converter warps
-// widen them into the same bf16 tile layout the MMAs read, so its ring of
-// bf16 tiles has two stages instead of three.
+// keeps the same three-stage ring of bf16 tiles.  TMA lands each 64-dim chunk
+// of a page's codes in the upper half of that chunk's 128-byte row slots
+// inside the stage, and the converter warps widen every (row, chunk) in place;
+// a page's 64 scales go to a small per-stage area.
 template <bool kFp8>
 struct Cfg {
   static constexpr int kThreads = kFp8 ? 256 + kConvThreads : 256;
-  static constexpr int kStages = kFp8 ? 2 : 3;
-  static constexpr int kSlots = kFp8 ? 2 : 0;
+  static constexpr int kStages = 3;
   static constexpr int kOffKV = 0;
   static constexpr int kOffP = kOffKV + kStages * kTileBytes;
-  static constexpr int kOffSlot = kOffP + kPBytes;
-  static constexpr int kOffBar = kOffSlot + kSlots * kFp8SlotBytes;
+  static constexpr int kOffScale = kOffP + kPBytes;                 // FP8: [stage][64] fp32
+  static constexpr int kOffBar = kOffScale + (kFp8 ? kStages * kPage * 4 : 0);
   static constexpr int kFull0 = 0, kEmpty0 = kStages, kQFull = 2 * kStages;
   static constexpr int kSFull0 = kQFull + 1, kSFull1 = kQFull + 2;
   static constexpr int kSFree0 = kQFull + 3, kSFree1 = kQFull + 4;
   static constexpr int kPFull = kQFull + 5, kPvDone = kQFull + 6, kOFull = kQFull + 7;
-  static constexpr int kSlotFull0 = kQFull + 8, kSlotEmpty0 = kSlotFull0 + kSlots;
-  static constexpr int kNumBars = kSlotEmpty0 + kSlots;
+  static constexpr int kLanded0 = kQFull + 8;                      // FP8: codes in the stage
+  static constexpr int kNumBars = kLanded0 + (kFp8 ? kStages : 0);
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem address + abort flag
   static constexpr int kSmemUsed = kOffMisc + 16;
   static constexpr int kSmemBytes = kSmemUsed + 1024;      // slack to align the base to 1024 B
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kOffP % 1024 == 0 && kOffSlot % 16 == 0, "alignment");
+  static_assert(kOffP % 1024 == 0 && kOffScale % 16 == 0, "alignment");
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -169,7 +166,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* skv = smem + C::kOffKV;
   uint8_t* sp = smem + C::kOffP;
-  uint8_t* sslot = smem + C::kOffSlot;  // FP8 cache only
+  float* sscale = reinterpret_cast<float*>(smem + C::kOffScale);  // FP8 cache only
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -200,9 +197,8 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar[kPFull], kSoftmaxThreads);
     mbar_init(&bar[kPvDone], 1);
     mbar_init(&bar[kOFull], 1);
-    for (int s = 0; s < C::kSlots; ++s) {
-      mbar_init(&bar[C::kSlotFull0 + s], 1);
-      mbar_init(&bar[C::kSlotEmpty0 + s], 1);
+    if constexpr (kFp8) {
+      for (int s = 0; s < kStages; ++s) mbar_init(&bar[C::kLanded0 + s], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -217,8 +213,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = *tmem_slot;
   // FP8 cache: 384 threads launched with 168 registers each; the softmax
   // warpgroup raises its budget to 232, the single-thread roles (warps 4-7)
-  // lower theirs to 56 and the converters to 96: 49152 of the 64512 in all.
-  constexpr int kNSlots = kFp8 ? C::kSlots : 1;  // keeps the bf16 instantiation well formed
+  // lower theirs to 56 and the converters to 128: 53248 of the 64512 in all.
   if constexpr (kFp8) {
     if (warp >= 4 && warp < kConvWarp0) setmaxnreg_dec<56>();
   }
@@ -226,122 +221,135 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   // The stage ring carries, per piece with pages, one entry for the query rows
   // followed by one entry per page; every role counts entries the same way.
   if (kFp8 && warp == kTmaWarp) {
-    // ------------------------------------------------------------ FP8 page producer
-    // Each page's codes (one 3-D box: 3 parts x 64 rows x 192 bytes) and its 64
-    // scales go to the next staging slot; the converter warps take it from there.
+    // ------------------------------------------------------------ FP8 producer
+    // Query rows as in the bf16 kernel (straight to the stage's full barrier).
+    // A page: for chunk c, one 128-byte x 64-row box whose x window is
+    // [64 c - 64, 64 c + 64) of the 576-byte row, so chunk c's codes land in
+    // bytes 64..127 of each 128-byte row slot of the tile's chunk c (bytes
+    // 0..63 get chunk c - 1's codes, or zeros for c = 0, and are overwritten by
+    // the converters); plus the page's 64 scales.  Both signal the stage's
+    // landed barrier; the converters signal full.
     if (lane == 0) {
+      prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_page);
-      int g = 0;
+      int entries = 0, last_q = -1;
+      uint32_t landed_parity = 0, landed_used = 0;  // per stage: page loads issued (mod 2), any
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (p.seqlens[pz.seq] > p.bt_stride * kPage) report(p.status, MLA_ERR_DEVICE_CHECK);
+        if (pz.npg == 0) continue;
         const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
-        for (int e = 0; e < pz.npg; ++e, ++g) {
-          const int slot = g % kNSlots, use = g / kNSlots;
+        for (int e = -1; e < pz.npg; ++e) {
+          const int stage = entries % kStages, use = entries / kStages;
           if (use > 0) {
-            ok = mbar_wait(&bar[C::kSlotEmpty0 + slot], (use - 1) & 1, abort_flag, kWaitLimitNs);
+            ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, kWaitLimitNs);
             if (!ok) break;
           }
-          uint8_t* dst = sslot + slot * kFp8SlotBytes;
-          int page = __ldg(bt + pz.pg0 + e);
-          // The tensor map bounds the codes load, but the untiled scale copy has
-          // no bounds: a page id outside the cache is reported and replaced.
-          if (page < 0 || page >= p.num_blocks) {
-            report(p.status, MLA_ERR_DEVICE_CHECK);
-            page = 0;
+          uint8_t* dst = skv + stage * kTileBytes;
+          if (e < 0) {
+            last_q = entries;
+            mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
+            const int qrow = pz.seq * p.rows + blockIdx.y * kRowsPerCta;
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
+          } else {
+            int page = __ldg(bt + pz.pg0 + e);
+            // The tensor map bounds the codes, but the untiled scale copy has no
+            // bounds: a page id outside the cache is reported and replaced.
+            if (page < 0 || page >= p.num_blocks) {
+              report(p.status, MLA_ERR_DEVICE_CHECK);
+              page = 0;
+            }
+            uint64_t* landed = &bar[C::kLanded0 + stage];
+            mbar_arrive_expect_tx(landed, kTileBytes + kPage * 4);
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_page, 64 * c - 64, page * kPage, landed);
+            bulk_load(sscale + stage * kPage, p.kscale + static_cast<int64_t>(page) * kPage,
+                      kPage * 4, landed);
+            landed_parity ^= 1u << stage;
+            landed_used |= 1u << stage;
           }
-          mbar_arrive_expect_tx(&bar[C::kSlotFull0 + slot], kFp8SlotBytes);
-          tma_load_3d(dst, &tm_page, 0, page * kPage, 0, &bar[C::kSlotFull0 + slot]);
-          bulk_load(dst + kFp8PageBytes, p.kscale + static_cast<int64_t>(page) * kPage, kPage * 4,
-                    &bar[C::kSlotFull0 + slot]);
+          ++entries;
         }
       }
-      for (int s = 0; s < kNSlots && s < g; ++s) {  // let every copy land (bounded)
-        const int n = g - 1 - s;
-        mbar_wait(&bar[C::kSlotFull0 + n % kNSlots], (n / kNSlots) & 1, abort_flag,
+      // Before leaving, let every copy this thread issued land (bounded): the
+      // last page load of each stage, and the last query load if no later
+      // entry reused its stage.
+      for (int s = 0; s < kStages; ++s)
+        if ((landed_used >> s) & 1)
+          mbar_wait(&bar[C::kLanded0 + s], ((landed_parity >> s) & 1) ^ 1, abort_flag,
+                    kWaitLimitNs);
+      if (last_q >= 0 && last_q >= entries - kStages)
+        mbar_wait(&bar[kFull0 + last_q % kStages], (last_q / kStages) & 1, abort_flag,
                   kWaitLimitNs);
-      }
     }
   } else if (kFp8 && warp >= kConvWarp0) {
     // ------------------------------------------------------------ FP8 converters
-    // Producers of the bf16 ring: the query rows of a piece by TMA (thread 0),
-    // and each page widened from its staging slot into the swizzled bf16 tile
-    // (row r, dims 16i..16i+15 per item).  Rows past the sequence's end are
-    // written as zeros, so stale codes or scales there never reach an MMA.
-    // The four warps decide together after a named barrier, so that a wait
-    // that gave up in one warp stops all of them at the same point.
-    if constexpr (kFp8) setmaxnreg_dec<96>();
+    // Widen each landed page in place: thread t owns row r = t % 64 of chunks
+    // t / 64, t / 64 + 2, ... (5 or 4 of the 9).  For each it reads the 64
+    // codes (bytes 64..127 of the row slot) into registers, then writes the 64
+    // bf16 values over the whole 128-byte slot, swizzled.  No other thread
+    // touches that slot, so reading before writing makes the in-place update
+    // safe.  The four 16-byte loads start at unit (r mod 4) and the eight 8-lane
+    // store phases cover 8 rows, so neither hits a bank more than twice.  Rows
+    // past the sequence's end are written as zeros, so stale codes or scales
+    // there never reach an MMA.  The four warps decide together after a named
+    // barrier, so that a wait that gave up in one warp stops all of them.
+    if constexpr (kFp8) setmaxnreg_dec<128>();
     const int ct = threadIdx.x - kConvWarp0 * 32;
-    int entries = 0, g = 0;
+    const int r = ct & 63, c0 = ct >> 6;
+    int entries = 0;
+    uint32_t landed_parity = 0;  // per stage: pages converted there (mod 2)
     for (int pc = 0; pc < npieces; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       if (pz.npg == 0) continue;
       const int L = p.seqlens[pz.seq];
+      entries += 1;  // the query entry goes straight to the consumers
       bool stop = false;
-      for (int e = -1; e < pz.npg; ++e) {
-        const int stage = entries % kStages, use = entries / kStages;
-        if (use > 0) warp_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag);
-        uint8_t* dst = skv + stage * kTileBytes;
-        if (e < 0) {
-          named_bar_sync(kConvBarrier, kConvThreads);
-          if (*abort_flag) { stop = true; break; }
-          if (ct == 0) {
-            const int qrow = pz.seq * p.rows + blockIdx.y * kRowsPerCta;
-            mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
-            for (int c = 0; c < kChunks; ++c)
-              tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
-          }
-        } else {
-          const int slot = g % kNSlots;
-          if (!*abort_flag)
-            warp_wait(&bar[C::kSlotFull0 + slot], (g / kNSlots) & 1, abort_flag);
-          named_bar_sync(kConvBarrier, kConvThreads);
-          if (*abort_flag) { stop = true; break; }
-          const uint8_t* src = sslot + slot * kFp8SlotBytes;
-          const float* scales = reinterpret_cast<const float*>(src + kFp8PageBytes);
-          const int valid = L - (pz.pg0 + e) * kPage;  // rows of this page inside the sequence
-          for (int it = ct; it < kPage * (kDqk / 16); it += kConvThreads) {
-            const int r = it / (kDqk / 16), i = it - r * (kDqk / 16);
+      for (int e = 0; e < pz.npg; ++e, ++entries) {
+        const int stage = entries % kStages;
+        const uint32_t parity = (landed_parity >> stage) & 1;
+        landed_parity ^= 1u << stage;
+        warp_wait(&bar[C::kLanded0 + stage], parity, abort_flag);  // gives up at once on abort
+        named_bar_sync(kConvBarrier, kConvThreads);
+        if (*abort_flag) { stop = true; break; }
+        uint8_t* tile = skv + stage * kTileBytes;
+        const bool row_ok = r < L - (pz.pg0 + e) * kPage;  // row inside the sequence
+        // 2^60 * scale as bf16x2 (a power of two: its fp32 bits end in 16 zeros)
+        const uint32_t f_lo = row_ok ? (__float_as_uint(sscale[stage * kPage + r] * 0x1p60f) >> 16) *
+                                           0x10001u
+                                     : 0u;
+        constexpr uint32_t f_hi = 0x5D805D80u;  // 2^60 in both halves
+        for (int c = c0; c < kChunks; c += 2) {
+          uint8_t* slot = tile + c * kChunkBytes + r * 128;
+          uint4 v[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            v[k] = *reinterpret_cast<const uint4*>(slot + 64 + 16 * ((k + r) & 3));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int kk = (k + r) & 3;  // v[k] holds dims 16 kk .. 16 kk + 15 of the chunk
             uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-            if (r < valid) {
-              const uint4 v = *reinterpret_cast<const uint4*>(
-                  src + (i / 12) * (kPage * kFp8PartBytes) + r * kFp8PartBytes + (i % 12) * 16);
-              // 2^60 * scale as bf16x2 (a power of two: its fp32 bits end in 16 zeros)
-              const uint32_t f_lo = (__float_as_uint(scales[r] * 0x1p60f) >> 16) * 0x10001u;
-              constexpr uint32_t f_hi = 0x5D805D80u;  // 2^60 in both halves
-              lo.x = e4m3x2_to_bf16x2(v.x, 0x1404u, f_hi, f_lo);
-              lo.y = e4m3x2_to_bf16x2(v.x, 0x3424u, f_hi, f_lo);
-              lo.z = e4m3x2_to_bf16x2(v.y, 0x1404u, f_hi, f_lo);
-              lo.w = e4m3x2_to_bf16x2(v.y, 0x3424u, f_hi, f_lo);
-              hi.x = e4m3x2_to_bf16x2(v.z, 0x1404u, f_hi, f_lo);
-              hi.y = e4m3x2_to_bf16x2(v.z, 0x3424u, f_hi, f_lo);
-              hi.z = e4m3x2_to_bf16x2(v.w, 0x1404u, f_hi, f_lo);
-              hi.w = e4m3x2_to_bf16x2(v.w, 0x3424u, f_hi, f_lo);
+            if (row_ok) {
+              lo.x = e4m3x2_to_bf16x2(v[k].x, 0x1404u, f_hi, f_lo);
+              lo.y = e4m3x2_to_bf16x2(v[k].x, 0x3424u, f_hi, f_lo);
+              lo.z = e4m3x2_to_bf16x2(v[k].y, 0x1404u, f_hi, f_lo);
+              lo.w = e4m3x2_to_bf16x2(v[k].y, 0x3424u, f_hi, f_lo);
+              hi.x = e4m3x2_to_bf16x2(v[k].z, 0x1404u, f_hi, f_lo);
+              hi.y = e4m3x2_to_bf16x2(v[k].z, 0x3424u, f_hi, f_lo);
+              hi.z = e4m3x2_to_bf16x2(v[k].w, 0x1404u, f_hi, f_lo);
+              hi.w = e4m3x2_to_bf16x2(v[k].w, 0x3424u, f_hi, f_lo);
             }
-            // dims 16i..16i+15: chunk i/4, 16-byte units 2(i%4) and 2(i%4)+1, swizzled by row
-            uint8_t* rowp = dst + (i >> 2) * kChunkBytes + r * 128;
-            const int u = 2 * (i & 3);
-            *reinterpret_cast<uint4*>(rowp + ((u ^ (r & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (r & 7)) << 4)) = hi;
+            *reinterpret_cast<uint4*>(slot + (((2 * kk) ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(slot + (((2 * kk + 1) ^ (r & 7)) << 4)) = hi;
           }
-          fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
-          named_bar_sync(kConvBarrier, kConvThreads);
-          if (ct == 0) {
-            mbar_arrive(&bar[C::kSlotEmpty0 + slot]);
-            mbar_arrive(&bar[kFull0 + stage]);
-          }
-          ++g;
         }
-        ++entries;
+        fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+        named_bar_sync(kConvBarrier, kConvThreads);
+        if (ct == 0) mbar_arrive(&bar[kFull0 + stage]);
       }
       if (stop) break;
-    }
-    if (ct == 0) {  // let the query copies land before leaving (bounded)
-      for (int s = 0; s < kStages && s < entries; ++s) {
-        const int n = entries - 1 - s;
-        mbar_wait(&bar[kFull0 + n % kStages], (n / kStages) & 1, abort_flag, kWaitLimitNs);
-      }
     }
   } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer

@@ -85,8 +85,8 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
-// FP8 (E4M3) cache, up to 64 query rows per sequence: tm_page8 is the codes viewed
-// as {192 bytes, rows, 3 parts} with a box of 192 x 64 x 3.
+// FP8 (E4M3) cache, up to 64 query rows per sequence: tm_page8 views the codes
+// as [rows, 576] bytes in boxes of 128 bytes x 64 rows; scales via p.kscale.
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
