@@ -134,13 +134,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
-// Hint: bring `bytes` (a multiple of 16) at a 16-byte aligned address into L2.
-__device__ __forceinline__ void l2_prefetch(const void* gaddr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)),
-               "r"(bytes)
-               : "memory");
-}
-
 // Barrier over `threads` threads (a multiple of 32) on hardware barrier `id` (1..15).
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
