@@ -308,7 +308,14 @@ def run_cuda(args, rank, local, world):
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(args.workload, seed=0)
     fp8 = args.kv == "fp8"
-    nbytes, flops = synth.algorithmic_work(inp, 580 if fp8 else 1152)
+    sparse_idx = None
+    if args.sparse_topk:
+        if fp8:
+            raise SystemExit("--sparse-topk runs on the bf16 cache")
+        sparse_idx = synth.make_sparse_indices(inp, args.sparse_topk, seed=0)
+        nbytes, flops = synth.sparse_algorithmic_work(inp, sparse_idx)
+    else:
+        nbytes, flops = synth.algorithmic_work(inp, 580 if fp8 else 1152)
     q = inp.q.to(dev)
     kc = inp.kcache.to(dev)
     bt = inp.block_table.to(dev)
@@ -325,6 +332,12 @@ def run_cuda(args, rank, local, world):
     ws = torch.empty((binding.workspace_size(b, s_q, h_q, num_workers),), dtype=torch.uint8,
                      device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    if sparse_idx is not None:
+        idx_d = sparse_idx.to(dev)
+        sp_workers, _ = binding.metadata_shape(b * s_q, h_q, 1)
+        sp_ws = torch.empty((binding.lib.mla_sparse_workspace_size(b, s_q, h_q, sparse_idx.shape[2],
+                                                                   sp_workers),),
+                            dtype=torch.uint8, device=dev)
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
     flush_max = torch.empty((), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -336,10 +349,15 @@ def run_cuda(args, rank, local, world):
         torch.amax(flush.view(torch.int32), dim=0, out=flush_max)
 
     def metadata():
+        if sparse_idx is not None:  # the sparse call runs its own scheduler
+            return None, None
         return binding.get_mla_metadata(sl, h_q, s_q, num_workers)
 
     def decode_call(md, ns):
-        if fp8:
+        if sparse_idx is not None:
+            binding.mla_decode_sparse(q, kc, bt, sl, idx_d, inp.scale, inp.causal, out=out, lse=lse,
+                                      workspace=sp_ws, device_status=status)
+        elif fp8:
             binding.mla_decode_kvcache_fp8(q, kc8, ks, bt, sl, 512, md, ns, inp.scale, inp.causal,
                                            out=out, lse=lse, workspace=ws, device_status=status)
         else:
@@ -372,8 +390,11 @@ def run_cuda(args, rank, local, world):
     g_step, g_meta, g_call = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step):
         step()
-    with torch.cuda.graph(g_meta):
-        md_g, ns_g = metadata()
+    if sparse_idx is None:
+        with torch.cuda.graph(g_meta):
+            md_g, ns_g = metadata()
+    else:  # the sparse call runs its own scheduler: nothing to capture apart
+        md_g, ns_g = None, None
     with torch.cuda.graph(g_call):
         decode_call(md_g, ns_g)
     for k in range(3):
@@ -413,7 +434,8 @@ def run_cuda(args, rank, local, world):
         flush_l2(k)
         e0, em, e1 = split_events[k]
         e0.record(stream)
-        g_meta.replay()
+        if sparse_idx is None:
+            g_meta.replay()
         em.record(stream)
         g_call.replay()
         e1.record(stream)
@@ -439,11 +461,21 @@ def run_cuda(args, rank, local, world):
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         dq, dbt, dsl = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
+        if sparse_idx is not None:
+            hidx = sparse_idx.pin_memory()
+            didx = torch.empty_like(idx_d)
 
         def e2e_step():
             dq.copy_(hq, non_blocking=True)
             dbt.copy_(hbt, non_blocking=True)
             dsl.copy_(hsl, non_blocking=True)
+            if sparse_idx is not None:
+                didx.copy_(hidx, non_blocking=True)
+                o, l = binding.mla_decode_sparse(dq, kc, dbt, dsl, didx, inp.scale, inp.causal,
+                                                 out=out, lse=lse, workspace=sp_ws)
+                hout.copy_(o, non_blocking=True)
+                hlse.copy_(l, non_blocking=True)
+                return
             md, ns = binding.get_mla_metadata(dsl, h_q, s_q, num_workers)
             if fp8:
                 o, l = binding.mla_decode_kvcache_fp8(dq, kc8, ks, dbt, dsl, 512, md, ns, inp.scale,
@@ -472,6 +504,8 @@ def run_cuda(args, rank, local, world):
         e2e_total = reduce_max(sum(a.elapsed_time(z) for a, z in e2e_ms) / 1e3, world, dev)
         e2e_bytes = reduce_sum(float(nbytes * n_e2e), world, dev)
         h2d = hq.numel() * hq.element_size() + hbt.numel() * 4 + hsl.numel() * 4
+        if sparse_idx is not None:
+            h2d += sparse_idx.numel() * 4
         d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
         e2e = {"value": e2e_bytes / e2e_total / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
@@ -502,6 +536,7 @@ def run_cuda(args, rank, local, world):
         "data": "synthetic (seeded N(0,1) bf16 q and latent cache, shuffled 64-token pages)",
         "config": workload_config(inp, {"parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                                         "num_workers": num_workers,
+                                        "sparse_topk": args.sparse_topk or None,
                                         "kv_cache": ("fp8: E4M3 codes + one power-of-two fp32 scale "
                                                      "per token (580 B per token)") if fp8 else
                                                     "bf16 (1152 B per token)"}),
@@ -509,14 +544,15 @@ def run_cuda(args, rank, local, world):
         "roofline_frac": max(t_hbm, t_tc) / (ms_per_step / 1e3),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak,
-                     "traffic": None if fp8 else recorded_traffic(args.workload),
+                     "traffic": None if (fp8 or sparse_idx is not None)
+                     else recorded_traffic(args.workload),
                      "kernel": "mla_decode_kvcache call (decode kernel + split combine)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s / 1.59 PFLOP/s"},
         "kernel_us": {"metadata": statistics.median(meta_ms) * 1e3,
                       "decode_call": statistics.median(decode_ms) * 1e3,
                       "step": statistics.median(step_ms) * 1e3},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": ((5 + (s_q > 1)) if sparse_idx is not None else 3) * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": t_wall,
     }
@@ -645,6 +681,9 @@ def main():
                          "up to 64 query rows per sequence)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
+    ap.add_argument("--sparse-topk", type=int, default=0,
+                    help="time the sparse decode with this many selected tokens per query "
+                         "position (seeded uniform picks; bf16 cache)")
     ap.add_argument("--no-append", action="store_true",
                     help="skip timing the latent-cache append")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,

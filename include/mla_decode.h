@@ -306,6 +306,48 @@ int mla_release_pages(const int32_t* release_mask, int32_t* block_table, int bt_
                       int32_t* cache_seqlens, int batch, int32_t* free_pages, int free_capacity,
                       int32_t* free_count, int32_t* device_status, void* stream);
 
+/*
+ * mla_sparse_workspace_size -- bytes of workspace mla_decode_sparse needs:
+ * the compacted index lists, the gathered rows (ceil(topk / 64) pages of 64
+ * rows x 1152 bytes per query position), the split metadata and partials of
+ * the decode over them.  num_workers: mla_metadata_shape(batch * s_q, h_q, 1).
+ * Returns 0 for invalid arguments.
+ */
+size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int num_workers);
+
+/*
+ * mla_decode_sparse -- sparse (top-k) decode given token indices.
+ *
+ * Dynamic sparse attention restricts each query to the most relevant cached
+ * tokens, reached by gathering them ("Boosting DeepSeek V3.2: Faster LLM
+ * Inference With FlashMLA", the paragraph on Dynamic Sparse Attention).  The
+ * selection is an input (choosing it needs an indexer with trained weights):
+ * indices: device int32 [batch, s_q, topk], logical token positions of
+ *          sequence i for query position j, shared by every head.  An entry t
+ *          is used when 0 <= t < L_i and, with causal, t <= L_i - s_q + j;
+ *          other entries (-1 padding) are skipped.  Each used entry is one
+ *          term, so a position listed twice counts twice.
+ * Over the used entries the result is mla_decode_kvcache's definition: out
+ * [batch, s_q, h_q, 512] bf16 and lse [batch, h_q, s_q] fp32; a query position
+ * with no used entry gets out = 0 and lse = -inf.
+ * num_workers: mla_metadata_shape(batch * s_q, h_q, 1).  workspace: at least
+ * mla_sparse_workspace_size(...) bytes, 256-byte aligned, contents need not
+ * be initialised.  The other arguments are as for mla_decode_kvcache.
+ * Requires topk <= 65536, batch * s_q <= 65536.  A used entry whose page lies
+ * outside the block-table row or the cache is read as a zero row and reported
+ * as MLA_ERR_DEVICE_CHECK in device_status.
+ * Launches: a compaction kernel and a gather kernel (each used entry's row is
+ * copied into workspace pages, one sequence per query position), then the
+ * scheduler, decode and combine kernels of mla_decode_kvcache over them, and
+ * (s_q > 1) a kernel that reorders lse.  No host synchronisation.
+ */
+int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
+                      const int32_t* block_table, int bt_stride, const int32_t* cache_seqlens,
+                      int batch, int s_q, int h_q, int d, int dv, const int32_t* indices,
+                      int topk, float softmax_scale, int causal, int num_workers,
+                      void* workspace, size_t workspace_bytes, void* out, float* lse,
+                      int32_t* device_status, void* stream);
+
 /* mla_error_string -- static text for a status code (never NULL). */
 const char* mla_error_string(int status);
 

@@ -31,7 +31,8 @@ STATIC_SCRATCH_BYTES = 48 << 20
 
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
            "mla_decode_kvcache_static_scratch", "mla_append_latent", "mla_release_pages",
-           "mla_append_latent_fp8", "mla_decode_kvcache_fp8", "mla_error_string", "mla_version")
+           "mla_append_latent_fp8", "mla_decode_kvcache_fp8", "mla_sparse_workspace_size",
+           "mla_decode_sparse", "mla_error_string", "mla_version")
 
 
 class MLAError(RuntimeError):
@@ -68,6 +69,11 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache_fp8.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, f32,
                                            i32, p, p, i32, p, sz, p, p, p, p]
     lib.mla_decode_kvcache_fp8.restype = i32
+    lib.mla_sparse_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.mla_sparse_workspace_size.restype = sz
+    lib.mla_decode_sparse.argtypes = [p, p, i64, p, i32, p, i32, i32, i32, i32, i32, p, i32, f32,
+                                      i32, i32, p, sz, p, p, p, p]
+    lib.mla_decode_sparse.restype = i32
     lib.mla_release_pages.argtypes = [p, p, i32, p, i32, p, i32, p, p, p]
     lib.mla_release_pages.restype = i32
     lib.mla_error_string.argtypes = [i32]
@@ -267,4 +273,41 @@ def mla_decode_kvcache_fp8(q: torch.Tensor, kcache8: torch.Tensor, kscale: torch
             int(bool(causal)), _ptr(tile_md), _ptr(num_splits), num_workers, _ptr(workspace),
             workspace.numel(), _ptr(out), _ptr(lse), _ptr(device_status), _stream_handle(dev))
         _check(rc, "mla_decode_kvcache_fp8")
+    return out, lse
+
+
+def mla_decode_sparse(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
+                      cache_seqlens: torch.Tensor, indices: torch.Tensor, softmax_scale: float,
+                      causal: bool = False, dv: int = D_V, out: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      device_status: torch.Tensor | None = None):
+    """Sparse decode: each query position attends to the cached tokens listed in
+    indices [b, s_q, topk] int32 (entries outside the sequence, or past the causal
+    limit, are skipped).  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q])."""
+    b, s_q, h_q, d = q.shape
+    dev = q.device
+    for t in (q, kcache, block_table, cache_seqlens, indices):
+        assert t.is_cuda and t.device == dev and t.is_contiguous()
+    assert q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
+    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
+    assert indices.dtype == torch.int32 and indices.dim() == 3
+    assert indices.shape[0] == b and indices.shape[1] == s_q
+    topk = indices.shape[2]
+    with torch.cuda.device(dev):
+        num_workers, _ = metadata_shape(b * s_q, h_q, 1)
+        if out is None:
+            out = torch.empty((b, s_q, h_q, dv), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+        need = int(lib.mla_sparse_workspace_size(b, s_q, h_q, topk, num_workers))
+        if need == 0:
+            raise MLAError(MLA_ERR_INVALID_ARG, "mla_sparse_workspace_size")
+        if workspace is None:
+            workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+        rc = lib.mla_decode_sparse(
+            _ptr(q), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.shape[1],
+            _ptr(cache_seqlens), b, s_q, h_q, d, dv, _ptr(indices), topk, float(softmax_scale),
+            int(bool(causal)), num_workers, _ptr(workspace), workspace.numel(), _ptr(out),
+            _ptr(lse), _ptr(device_status), _stream_handle(dev))
+        _check(rc, "mla_decode_sparse")
     return out, lse

@@ -352,6 +352,89 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
 }
 
+size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int num_workers) {
+  if (batch < 1 || s_q < 1 || h_q < 1 || topk < 1 || num_workers < 1) return 0;
+  const size_t pos = static_cast<size_t>(batch) * s_q;
+  const size_t ppp = (static_cast<size_t>(topk) + mla::kPage - 1) / mla::kPage;
+  const size_t dec = mla_workspace_size(static_cast<int>(pos), 1, h_q, mla::kDv, num_workers);
+  if (dec == 0) return 0;
+  return round_up(pos * topk * 4, 256) + round_up(pos * 4, 256) + round_up(pos * ppp * 4, 256) +
+         round_up(static_cast<size_t>(num_workers) * MLA_MD_STRIDE * 4, 256) +
+         round_up((pos + 1) * 4, 256) + round_up(pos * h_q * 4, 256) + dec +
+         pos * ppp * mla::kPage * mla::kDqk * 2;
+}
+
+int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
+                      const int32_t* block_table, int bt_stride, const int32_t* cache_seqlens,
+                      int batch, int s_q, int h_q, int d, int dv, const int32_t* indices,
+                      int topk, float softmax_scale, int causal, int num_workers,
+                      void* workspace, size_t workspace_bytes, void* out, float* lse,
+                      int32_t* device_status, void* stream) {
+  if (q == nullptr || kcache == nullptr || block_table == nullptr || cache_seqlens == nullptr ||
+      indices == nullptr || workspace == nullptr || out == nullptr || lse == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (d != mla::kDqk || dv != mla::kDv) return MLA_ERR_UNSUPPORTED;
+  if (batch < 1 || s_q < 1 || h_q < 1 || bt_stride < 1 || topk < 1 || topk > 65536 ||
+      num_workers < 1 || num_workers > (1 << 20) || (causal != 0 && causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(h_q) > 65536) return MLA_ERR_UNSUPPORTED;
+  if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+  const int64_t pos = static_cast<int64_t>(batch) * s_q;
+  const int64_t ppp = (topk + mla::kPage - 1) / mla::kPage;
+  if (pos > 65536 || pos * ppp * mla::kPage >= (int64_t(1) << 31) ||
+      pos * h_q >= (int64_t(1) << 31))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+      !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_sparse_workspace_size(batch, s_q, h_q, topk, num_workers);
+  if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
+
+  char* w = static_cast<char*>(workspace);
+  auto take = [&w](size_t bytes) {
+    char* r = w;
+    w += round_up(bytes, 256);
+    return r;
+  };
+  mla::SparseParams sp{};
+  sp.indices = indices;
+  sp.seqlens = cache_seqlens;
+  sp.block_table = block_table;
+  sp.kcache = kcache;
+  sp.comp = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos) * topk * 4));
+  sp.counts = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos) * 4));
+  sp.comp_bt = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos * ppp) * 4));
+  int32_t* tile_md = reinterpret_cast<int32_t*>(take(static_cast<size_t>(num_workers) * MLA_MD_STRIDE * 4));
+  int32_t* num_splits = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos + 1) * 4));
+  float* lse_pos = reinterpret_cast<float*>(take(static_cast<size_t>(pos) * h_q * 4));
+  const size_t dec_bytes = mla_workspace_size(static_cast<int>(pos), 1, h_q, mla::kDv, num_workers);
+  void* dec_ws = take(dec_bytes);
+  sp.comp_cache = w;  // the rest: the gathered pages
+  sp.status = device_status;
+  sp.bt_stride = bt_stride;
+  sp.num_blocks = num_blocks;
+  sp.batch = batch;
+  sp.s_q = s_q;
+  sp.topk = topk;
+  sp.causal = causal;
+  sp.pages_per_pos = static_cast<int>(ppp);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mla::launch_sparse_prepare(sp, st) != cudaSuccess) return MLA_ERR_CUDA;
+  int rc = mla_get_metadata(sp.counts, static_cast<int>(pos), h_q, 1, tile_md, num_splits,
+                            num_workers, stream);
+  if (rc != MLA_OK) return rc;
+  rc = mla_decode_kvcache(q, sp.comp_cache, pos * ppp, sp.comp_bt, static_cast<int>(ppp),
+                          sp.counts, static_cast<int>(pos), 1, h_q, d, dv, softmax_scale, 0,
+                          tile_md, num_splits, num_workers, dec_ws, dec_bytes, out,
+                          s_q > 1 ? lse_pos : lse, device_status, stream);
+  if (rc != MLA_OK) return rc;
+  if (s_q > 1 && mla::launch_sparse_lse(lse_pos, lse, batch, s_q, h_q, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
 }  // extern "C"
 
 namespace {

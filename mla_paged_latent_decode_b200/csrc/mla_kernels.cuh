@@ -77,7 +77,25 @@ struct ReleaseParams {
   int batch, free_capacity;
 };
 
+// Sparse decode: compaction of used indices and gather of their rows (mla_sparse.cu).
+struct SparseParams {
+  const int32_t* indices;      // [batch * s_q, topk]
+  const int32_t* seqlens;      // [batch]
+  const int32_t* block_table;  // [batch, bt_stride]
+  const void* kcache;          // [num_blocks * 64, 576] bf16
+  int32_t* comp;               // workspace [batch * s_q, topk]: used entries, in order
+  int32_t* counts;             // workspace [batch * s_q]
+  int32_t* comp_bt;            // workspace [batch * s_q, pages_per_pos]
+  void* comp_cache;            // workspace [batch * s_q * pages_per_pos * 64, 576] bf16
+  int32_t* status;             // nullable
+  int64_t bt_stride, num_blocks;
+  int batch, s_q, topk, causal, pages_per_pos;
+};
+
 // Launchers (return cudaGetLastError() of their launch).
+cudaError_t launch_sparse_prepare(const SparseParams& p, cudaStream_t stream);
+cudaError_t launch_sparse_lse(const float* lse_pos, float* lse, int batch, int s_q, int h_q,
+                              cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, bool fp8, cudaStream_t stream);
 cudaError_t launch_release(const ReleaseParams& p, cudaStream_t stream);
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,

@@ -185,3 +185,41 @@ def algorithmic_work(inp: DecodeInputs, kv_bytes_per_token: int = D_QK * 2) -> t
             pairs += max(0, min(vis, L))
     flops = 2 * (D_QK + D_V) * h_q * pairs
     return nbytes, flops
+
+
+def make_sparse_indices(inp: DecodeInputs, topk: int, seed: int = 0, pad_frac: float = 0.0):
+    """indices [b, s_q, topk] int32 for the sparse decode: for each query
+    position, min(topk, L) distinct positions drawn uniformly from [0, L) in
+    random order, the rest -1.  With pad_frac > 0 that fraction of the drawn
+    entries is replaced by -1 or by positions past the sequence's end."""
+    gen = torch.Generator().manual_seed(seed)
+    b, s_q = inp.batch, inp.s_q
+    idx = torch.full((b, s_q, topk), -1, dtype=torch.int32)
+    for i, L in enumerate(inp.cache_seqlens.tolist()):
+        for j in range(s_q):
+            k = min(topk, L)
+            if k > 0:
+                idx[i, j, :k] = torch.randperm(L, generator=gen)[:k].to(torch.int32)
+    if pad_frac > 0:
+        drop = torch.rand((b, s_q, topk), generator=gen) < pad_frac
+        far = torch.rand((b, s_q, topk), generator=gen) < 0.5
+        idx = torch.where(drop & far, torch.full_like(idx, 1 << 30), idx)
+        idx = torch.where(drop & ~far, torch.full_like(idx, -1), idx)
+    return idx.contiguous()
+
+
+def sparse_algorithmic_work(inp: DecodeInputs, indices: torch.Tensor) -> tuple[int, int]:
+    """(bytes, flops) of one sparse decode call: every used entry's cached row
+    once (1152 bytes), q in, out and lse out, and the index lists; 2 * (576 +
+    512) flops per (head, used entry)."""
+    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
+    lens = inp.cache_seqlens.tolist()
+    used = 0
+    for i in range(b):
+        for j in range(s_q):
+            lim = min(lens[i] - s_q + j + 1, lens[i]) if inp.causal else lens[i]
+            row = indices[i, j]
+            used += int(((row >= 0) & (row < lim)).sum())
+    nbytes = (used * D_QK * 2 + b * s_q * h_q * (D_QK * 2 + D_V * 2) + b * h_q * s_q * 4
+              + indices.numel() * 4)
+    return nbytes, 2 * (D_QK + D_V) * h_q * used
