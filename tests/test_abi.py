@@ -139,3 +139,79 @@ def test_release_host_validation():
     for kw in (dict(mask=0), dict(bt=0), dict(sl=0), dict(fp=0), dict(fc=0), dict(stride=0),
                dict(batch=0), dict(cap=0)):
         assert call(**kw) == binding.MLA_ERR_INVALID_ARG
+
+
+def _fp8_decode_raw(**kw):
+    args = dict(q=1 << 12, kcache=1 << 12, kscale=1 << 12, num_blocks=4, block_table=1 << 12,
+                bt_stride=3, cache_seqlens=1 << 12, batch=2, s_q=1, h_q=16, d=576, dv=512,
+                scale=0.07, causal=0, tile_md=1 << 12, num_splits=1 << 12, num_workers=148,
+                workspace=1 << 12, workspace_bytes=1 << 30, out=1 << 12, lse=1 << 12)
+    args.update(kw)
+    v = ctypes.c_void_p
+    return binding.lib.mla_decode_kvcache_fp8(
+        v(args["q"]), v(args["kcache"]), v(args["kscale"]), args["num_blocks"],
+        v(args["block_table"]), args["bt_stride"], v(args["cache_seqlens"]), args["batch"],
+        args["s_q"], args["h_q"], args["d"], args["dv"], args["scale"], args["causal"],
+        v(args["tile_md"]), v(args["num_splits"]), args["num_workers"], v(args["workspace"]),
+        args["workspace_bytes"], v(args["out"]), v(args["lse"]), v(0), v(0))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kscale=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(kcache=0), binding.MLA_ERR_INVALID_ARG),
+    (dict(kscale=(1 << 12) + 4), binding.MLA_ERR_INVALID_ARG),
+    (dict(h_q=128), binding.MLA_ERR_UNSUPPORTED),      # more than 64 query rows
+    (dict(s_q=2, h_q=64), binding.MLA_ERR_UNSUPPORTED),
+    (dict(d=512), binding.MLA_ERR_UNSUPPORTED),
+    (dict(causal=3), binding.MLA_ERR_INVALID_ARG),
+    (dict(workspace_bytes=64), binding.MLA_ERR_INVALID_ARG),
+])
+def test_fp8_decode_host_validation(kw, code):
+    assert _fp8_decode_raw(**kw) == code
+
+
+def test_fp8_append_host_validation():
+    v = ctypes.c_void_p
+    ok = dict(rows=1 << 12, s_new=1, kc=1 << 12, ks=1 << 12, nb=4, bt=1 << 12, stride=3,
+              sl=1 << 12, batch=2, fp=1 << 12, cap=4, fc=1 << 12)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return binding.lib.mla_append_latent_fp8(
+            v(a["rows"]), a["s_new"], v(a["kc"]), v(a["ks"]), a["nb"], v(a["bt"]), a["stride"],
+            v(a["sl"]), a["batch"], v(a["fp"]), a["cap"], v(a["fc"]), v(0), v(0))
+    for kw in (dict(ks=0), dict(kc=0), dict(rows=0), dict(ks=(1 << 12) + 8), dict(s_new=0),
+               dict(batch=0), dict(nb=1 << 25)):
+        assert call(**kw) == binding.MLA_ERR_INVALID_ARG, kw
+
+
+def test_sparse_workspace_size_and_validation():
+    lib = binding.lib
+    pos, topk, h_q, W = 2 * 3, 100, 16, 148
+    ppp = -(-topk // 64)
+    r = lambda n: -(-n // 256) * 256
+    dec = binding.workspace_size(pos, 1, h_q, W)
+    expect = (r(pos * topk * 4) + r(pos * 4) + r(pos * ppp * 4) + r(W * 8 * 4) + r((pos + 1) * 4)
+              + r(pos * h_q * 4) + dec + pos * ppp * 64 * 576 * 2)
+    assert lib.mla_sparse_workspace_size(2, 3, h_q, topk, W) == expect
+    assert lib.mla_sparse_workspace_size(2, 3, h_q, 0, W) == 0
+    v = ctypes.c_void_p
+    ok = dict(q=1 << 12, kc=1 << 12, nb=4, bt=1 << 12, stride=3, sl=1 << 12, batch=2, s_q=3,
+              h_q=16, d=576, dv=512, idx=1 << 12, topk=100, scale=0.07, causal=0, W=148,
+              ws=1 << 12, wsb=1 << 40, out=1 << 12, lse=1 << 12)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.mla_decode_sparse(
+            v(a["q"]), v(a["kc"]), a["nb"], v(a["bt"]), a["stride"], v(a["sl"]), a["batch"],
+            a["s_q"], a["h_q"], a["d"], a["dv"], v(a["idx"]), a["topk"], a["scale"], a["causal"],
+            a["W"], v(a["ws"]), a["wsb"], v(a["out"]), v(a["lse"]), v(0), v(0))
+    for kw, code in ((dict(idx=0), binding.MLA_ERR_INVALID_ARG),
+                     (dict(topk=0), binding.MLA_ERR_INVALID_ARG),
+                     (dict(topk=65537), binding.MLA_ERR_INVALID_ARG),
+                     (dict(d=512), binding.MLA_ERR_UNSUPPORTED),
+                     (dict(ws=(1 << 12) + 16), binding.MLA_ERR_INVALID_ARG),
+                     (dict(wsb=1000), binding.MLA_ERR_INVALID_ARG),
+                     (dict(batch=70000), binding.MLA_ERR_INVALID_ARG),
+                     (dict(scale=float("inf")), binding.MLA_ERR_INVALID_ARG)):
+        assert call(**kw) == code, kw
