@@ -33,6 +33,12 @@
 // producer, warps 5 and 7 QK^T issuers for even and odd pages (warp 5 also
 // allocates TMEM), warp 6 PV issuer.
 //
+// FP8 cache (template argument kFp8): the same kernel over E4M3 codes with one
+// power-of-two scale per token.  The TMA warp lands each page chunk's codes in
+// the upper half of that chunk's 128-byte row slots inside the bf16 stage, and
+// four more warps (384 threads) widen them in place into the bf16 tile, exactly;
+// the MMAs, softmax and epilogue are unchanged.
+//
 // The method follows "FlashMLA: Revolutionizing Efficient Decoding...",
 // sections 4.2.1-4.2.3 (TMA prefetch of 64-row latent blocks into shared
 // memory, tensor cores for QK^T and PV, softmax fused into the kernel),
