@@ -100,6 +100,12 @@ def _check(code: int, what: str):
         raise MLAError(code, what)
 
 
+def _require(ok: bool, what: str):
+    """Argument check that stays on under `python -O` (unlike assert)."""
+    if not ok:
+        raise ValueError(f"invalid argument: {what}")
+
+
 def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
@@ -124,8 +130,10 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, h_q: int, s_q: int,
                      num_workers: int | None = None):
     """Split-KV tile scheduler.  Returns (tile_md [W, 8] int32, num_splits [b + 1] int32),
     both on cache_seqlens' device, produced on the current stream."""
-    assert cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32
-    assert cache_seqlens.dim() == 1 and cache_seqlens.is_contiguous()
+    _require(cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32,
+             "cache_seqlens must be int32 on a CUDA device")
+    _require(cache_seqlens.dim() == 1 and cache_seqlens.is_contiguous(),
+             "cache_seqlens must be 1-D and contiguous")
     dev = cache_seqlens.device
     b = cache_seqlens.numel()
     with torch.cuda.device(dev):
@@ -149,11 +157,16 @@ def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch
     b, s_q, h_q, d = q.shape
     dev = q.device
     for t in (q, kcache, block_table, cache_seqlens, tile_md, num_splits):
-        assert t.is_cuda and t.device == dev and t.is_contiguous()
-    assert q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
-    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
-    assert kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d
-    assert block_table.dim() == 2 and block_table.shape[0] == b
+        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
+                 "every tensor must be contiguous on q's CUDA device")
+    _require(q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16,
+             "q and kcache must be bf16")
+    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
+             "block_table and cache_seqlens must be int32")
+    _require(kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d,
+             "kcache must be [num_blocks, 64, 576]")
+    _require(block_table.dim() == 2 and block_table.shape[0] == b,
+             "block_table must be [batch, max_pages]")
     num_workers = tile_md.shape[0]
     with torch.cuda.device(dev):
         if out is None:
@@ -174,9 +187,11 @@ def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch
 
 def _check_state(block_table, cache_seqlens, free_pages, free_count, dev):
     for t in (block_table, cache_seqlens, free_pages, free_count):
-        assert t.is_cuda and t.device == dev and t.is_contiguous() and t.dtype == torch.int32
-    assert block_table.dim() == 2 and block_table.shape[0] == cache_seqlens.numel()
-    assert free_count.numel() == 1
+        _require(t.is_cuda and t.device == dev and t.is_contiguous() and t.dtype == torch.int32,
+                 "page-state tensors must be contiguous int32 on one CUDA device")
+    _require(block_table.dim() == 2 and block_table.shape[0] == cache_seqlens.numel(),
+             "block_table must be [batch, max_pages]")
+    _require(free_count.numel() == 1, "free_count must hold one int32")
 
 
 def append_latent(rows: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
@@ -187,11 +202,14 @@ def append_latent(rows: torch.Tensor, kcache: torch.Tensor, block_table: torch.T
     cache_seqlens and free_count in place, on the current stream."""
     b, s_new, d = rows.shape
     dev = rows.device
-    assert rows.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
-    assert rows.is_contiguous() and kcache.is_contiguous() and kcache.device == dev
-    assert kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d == D_QK
+    _require(rows.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16,
+             "rows and kcache must be bf16")
+    _require(rows.is_contiguous() and kcache.is_contiguous() and kcache.device == dev,
+             "rows and kcache must be contiguous on one device")
+    _require(kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d == D_QK,
+             "kcache must be [num_blocks, 64, 576] and rows [batch, s_new, 576]")
     _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
-    assert cache_seqlens.numel() == b
+    _require(cache_seqlens.numel() == b, "cache_seqlens must have one entry per sequence")
     with torch.cuda.device(dev):
         _check(lib.mla_append_latent(_ptr(rows), s_new, _ptr(kcache), kcache.shape[0],
                                      _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
@@ -207,8 +225,10 @@ def release_pages(release_mask: torch.Tensor, block_table: torch.Tensor,
     set its length to 0 (in place, on the current stream)."""
     dev = cache_seqlens.device
     _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
-    assert release_mask.dtype == torch.int32 and release_mask.device == dev
-    assert release_mask.is_contiguous() and release_mask.numel() == cache_seqlens.numel()
+    _require(release_mask.dtype == torch.int32 and release_mask.device == dev,
+             "release_mask must be int32 on the cache's device")
+    _require(release_mask.is_contiguous() and release_mask.numel() == cache_seqlens.numel(),
+             "release_mask must be contiguous, one entry per sequence")
     with torch.cuda.device(dev):
         _check(lib.mla_release_pages(_ptr(release_mask), _ptr(block_table), block_table.shape[1],
                                      _ptr(cache_seqlens), cache_seqlens.numel(), _ptr(free_pages),
@@ -225,13 +245,17 @@ def append_latent_fp8(rows: torch.Tensor, kcache8: torch.Tensor, kscale: torch.T
     codes (kcache8 [nblk, 64, 576] uint8) and per-token scales (kscale [nblk, 64] fp32)."""
     b, s_new, d = rows.shape
     dev = rows.device
-    assert rows.dtype == torch.bfloat16 and rows.is_contiguous() and d == D_QK
-    assert kcache8.dtype == torch.uint8 and kcache8.is_contiguous() and kcache8.device == dev
-    assert kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == D_QK
-    assert kscale.dtype == torch.float32 and kscale.is_contiguous()
-    assert tuple(kscale.shape) == tuple(kcache8.shape[:2])
+    _require(rows.dtype == torch.bfloat16 and rows.is_contiguous() and d == D_QK,
+             "rows must be contiguous bf16 [batch, s_new, 576]")
+    _require(kcache8.dtype == torch.uint8 and kcache8.is_contiguous() and kcache8.device == dev,
+             "kcache8 must be contiguous uint8 on the rows' device")
+    _require(kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == D_QK,
+             "kcache8 must be [num_blocks, 64, 576]")
+    _require(kscale.dtype == torch.float32 and kscale.is_contiguous(),
+             "kscale must be contiguous fp32")
+    _require(tuple(kscale.shape) == tuple(kcache8.shape[:2]), "kscale must be [num_blocks, 64]")
     _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
-    assert cache_seqlens.numel() == b
+    _require(cache_seqlens.numel() == b, "cache_seqlens must have one entry per sequence")
     with torch.cuda.device(dev):
         _check(lib.mla_append_latent_fp8(_ptr(rows), s_new, _ptr(kcache8), _ptr(kscale),
                                          kcache8.shape[0], _ptr(block_table), block_table.shape[1],
@@ -253,11 +277,16 @@ def mla_decode_kvcache_fp8(q: torch.Tensor, kcache8: torch.Tensor, kscale: torch
     b, s_q, h_q, d = q.shape
     dev = q.device
     for t in (q, kcache8, kscale, block_table, cache_seqlens, tile_md, num_splits):
-        assert t.is_cuda and t.device == dev and t.is_contiguous()
-    assert q.dtype == torch.bfloat16 and kcache8.dtype == torch.uint8
-    assert kscale.dtype == torch.float32 and tuple(kscale.shape) == tuple(kcache8.shape[:2])
-    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
-    assert kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == d
+        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
+                 "every tensor must be contiguous on q's CUDA device")
+    _require(q.dtype == torch.bfloat16 and kcache8.dtype == torch.uint8,
+             "q must be bf16 and kcache8 uint8")
+    _require(kscale.dtype == torch.float32 and tuple(kscale.shape) == tuple(kcache8.shape[:2]),
+             "kscale must be fp32 [num_blocks, 64]")
+    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
+             "block_table and cache_seqlens must be int32")
+    _require(kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == d,
+             "kcache8 must be [num_blocks, 64, 576]")
     num_workers = tile_md.shape[0]
     with torch.cuda.device(dev):
         if out is None:
@@ -287,11 +316,16 @@ def mla_decode_sparse(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.
     b, s_q, h_q, d = q.shape
     dev = q.device
     for t in (q, kcache, block_table, cache_seqlens, indices):
-        assert t.is_cuda and t.device == dev and t.is_contiguous()
-    assert q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16
-    assert block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32
-    assert indices.dtype == torch.int32 and indices.dim() == 3
-    assert indices.shape[0] == b and indices.shape[1] == s_q
+        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
+                 "every tensor must be contiguous on q's CUDA device")
+    _require(q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16,
+             "q and kcache must be bf16")
+    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
+             "block_table and cache_seqlens must be int32")
+    _require(indices.dtype == torch.int32 and indices.dim() == 3,
+             "indices must be int32 [batch, s_q, topk]")
+    _require(indices.shape[0] == b and indices.shape[1] == s_q,
+             "indices must be [batch, s_q, topk]")
     topk = indices.shape[2]
     with torch.cuda.device(dev):
         num_workers, _ = metadata_shape(b * s_q, h_q, 1)

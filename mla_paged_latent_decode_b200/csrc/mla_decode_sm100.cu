@@ -47,6 +47,8 @@
 // warps of its own.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "mla_kernels.cuh"
 #include "sm100_ptx.cuh"
 
@@ -700,16 +702,16 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // per device: attribute set
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (!configured[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(mla_decode_sm100_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
   cudaLaunchConfig_t cfg = {};
@@ -729,16 +731,16 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
 
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
                               const DecodeParams& p, int num_workers, cudaStream_t stream) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // per device: attribute set
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (!configured[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(mla_decode_sm100_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<true>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
   cudaLaunchConfig_t cfg = {};
