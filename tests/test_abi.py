@@ -215,3 +215,18 @@ def test_sparse_workspace_size_and_validation():
                      (dict(batch=70000), binding.MLA_ERR_INVALID_ARG),
                      (dict(scale=float("inf")), binding.MLA_ERR_INVALID_ARG)):
         assert call(**kw) == code, kw
+
+
+def test_binding_rejects_bad_tensors_before_any_call():
+    # checks that stay on under `python -O`: CPU tensors and wrong dtypes raise ValueError
+    import torch
+    with pytest.raises(ValueError):
+        binding.get_mla_metadata(torch.zeros(3, dtype=torch.int32), 16, 1)
+    with pytest.raises(ValueError):
+        binding.get_mla_metadata(torch.zeros(3, dtype=torch.int64), 16, 1)
+    q = torch.zeros((1, 1, 16, 576), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.mla_decode_sparse(q, torch.zeros((1, 64, 576), dtype=torch.bfloat16),
+                                  torch.zeros((1, 1), dtype=torch.int32),
+                                  torch.ones(1, dtype=torch.int32),
+                                  torch.zeros((1, 1, 4), dtype=torch.int32), 0.07)
