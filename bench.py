@@ -27,6 +27,13 @@ with an event between them, give the scheduler's time and the decode call's
 (decode kernel + split combine), which the roofline uses; there the decode
 starts only after the scheduler has finished.
 
+The line also carries `workloads`: every configuration (tiny, dsv3_decode,
+varlen_h16, spec_causal, skewed_long) measured in the same run, bf16 cache,
+default launch configuration: median / p10 / p90 of the step and of the decode
+call over --sweep-reps graph replays, each after an L2 flush, with bytes, flops
+and the roofline of each.  NVML clock samples cover the timed steps through
+the end of that sweep (`clocks`); the timed steps' own are `clocks_timed_region`.
+
 `--impl reference` times the fp64 CPU oracle on this host instead (bounded
 samples of the same workload), printing the same JSON line with
 "impl": "reference".
@@ -108,7 +115,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._period = period_s
@@ -157,11 +164,16 @@ class ClockSampler:
         if self._handle is not None:
             self._thread.join()
 
-    def summary(self):
-        if not self.samples:
+    def mark(self) -> int:
+        """Number of samples taken so far (to tell the timed region's apart)."""
+        return len(self.samples)
+
+    def summary(self, first: int = 0, last: int | None = None):
+        xs = self.samples[first:last]
+        if not xs:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(xs), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(xs), "reasons": sorted(self.reasons), "samples": len(xs)}
 
 
 def workload_config(inp, extra=None):
@@ -264,6 +276,106 @@ def reduce_sum(value: float, world: int, device) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def percentiles(xs):
+    """(median, p10, p90) of a list of numbers."""
+    ys = sorted(xs)
+    n = len(ys)
+
+    def at(f):
+        k = min(n - 1, max(0, int(round(f * (n - 1)))))
+        return ys[k]
+    return statistics.median(ys), at(0.10), at(0.90)
+
+
+def roofline_of(nbytes, flops, seconds, peaks):
+    """The bound (whichever of bytes / HBM peak and flops / bf16 peak is longer)
+    and the achieved rate against it for a call taking `seconds`."""
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved, peak, unit, bound = nbytes / seconds / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    else:
+        achieved, peak, unit, bound = flops / seconds / 1e12, peaks["bf16_tflops"], "TFLOP/s", \
+            "tensor"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "bound_us": max(t_hbm, t_tc) * 1e6}
+
+
+def measure_workload(name, dev, stream, flush_l2, reps, peaks):
+    """Every configuration of the decode measured the same way as the headline
+    one (bf16 cache, default launch configuration): `reps` graph replays of the
+    whole step and of the decode call alone, each after an L2 flush."""
+    from mla_paged_latent_decode_b200 import binding
+    inp = synth.make_inputs(name, seed=0)
+    nbytes, flops = synth.algorithmic_work(inp)
+    q, kc = inp.q.to(dev), inp.kcache.to(dev)
+    bt, sl = inp.block_table.to(dev), inp.cache_seqlens.to(dev)
+    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
+    nw, _ = binding.metadata_shape(b, h_q, s_q)
+    out = torch.empty((b, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    ws = torch.empty((binding.workspace_size(b, s_q, h_q, nw),), dtype=torch.uint8, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def call(md, ns):
+        binding.mla_decode_kvcache(q, kc, bt, sl, 512, md, ns, inp.scale, inp.causal, out=out,
+                                   lse=lse, workspace=ws, device_status=status)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            call(*binding.get_mla_metadata(sl, h_q, s_q, nw))
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g_step, g_meta, g_call = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        call(*binding.get_mla_metadata(sl, h_q, s_q, nw))
+    with torch.cuda.graph(g_meta):
+        md_g, ns_g = binding.get_mla_metadata(sl, h_q, s_q, nw)
+    with torch.cuda.graph(g_call):
+        call(md_g, ns_g)
+    for k in range(3):
+        flush_l2(k)
+        g_step.replay()
+    torch.cuda.synchronize(dev)
+    step_ev, call_ev = [], []
+    for k in range(reps):
+        flush_l2(k)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_step.replay()
+        e1.record(stream)
+        step_ev.append((e0, e1))
+    for k in range(reps):
+        flush_l2(k)
+        g_meta.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_call.replay()
+        e1.record(stream)
+        call_ev.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    del g_step, g_meta, g_call
+    if int(status.item()) != 0:
+        raise RuntimeError(f"{name}: device status {int(status.item())}")
+    step_us = percentiles([a.elapsed_time(z) * 1e3 for a, z in step_ev])
+    call_us = percentiles([a.elapsed_time(z) * 1e3 for a, z in call_ev])
+    kernel = "pair" if s_q * h_q > 64 else "single-CTA"
+    return {
+        "workload": f"{name}: {inp.workload.description}", "kernel": kernel, "num_workers": nw,
+        "pieces": None, "bytes": nbytes, "flops": flops,
+        "decode_call_us": call_us[0], "decode_call_us_p10": call_us[1],
+        "decode_call_us_p90": call_us[2],
+        "step_us": step_us[0], "step_us_p10": step_us[1], "step_us_p90": step_us[2],
+        "tb_s_step": nbytes / (step_us[0] * 1e-6) / 1e12,
+        "tflops_step": flops / (step_us[0] * 1e-6) / 1e12,
+        "roofline": roofline_of(nbytes, flops, call_us[0] * 1e-6, peaks),
+        "roofline_frac_step": roofline_of(nbytes, flops, step_us[0] * 1e-6, peaks)["frac"],
+        "reps": reps,
+    }
 
 
 # ----------------------------------------------------------------------------- arms
@@ -406,16 +518,19 @@ def run_cuda(args, rank, local, world):
               for _ in range(args.steps)]
     barrier(world, dev)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        t_wall0 = time.perf_counter()
-        for k in range(args.steps):
-            flush_l2(k)
-            e0, e1 = events[k]
-            e0.record(stream)
-            g_step.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        t_wall = time.perf_counter() - t_wall0
+    # NVML samples from here to the end of the per-workload sweep; the timed
+    # region's own samples are reported apart
+    clocks = ClockSampler(local).__enter__()
+    t_wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush_l2(k)
+        e0, e1 = events[k]
+        e0.record(stream)
+        g_step.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter() - t_wall0
+    timed_samples = clocks.mark()
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     step_ms = [e0.elapsed_time(e1) for e0, e1 in events]
@@ -514,21 +629,27 @@ def run_cuda(args, rank, local, world):
 
     append = None if args.no_append else measure_append(inp, dev, stream, flush_l2, fp8=fp8)
 
+    peaks, peak_kind = load_peaks()
+    workloads = None
+    if not (args.no_workloads or fp8 or sparse_idx is not None):
+        # every configuration, bf16 cache, from the same run (the headline one included)
+        workloads = {}
+        for name in synth.WORKLOADS:
+            workloads[name] = measure_workload(name, dev, stream, flush_l2, args.sweep_reps, peaks)
+            torch.cuda.empty_cache()
+    clocks.__exit__(None, None, None)
+
     if rank != 0:
         return None
-    peaks, peak_kind = load_peaks()
     ms_per_step = total_s / args.steps * 1e3
     value = all_bytes / total_s / 1e12
     tflops = all_flops / total_s / 1e12
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    if bound == "hbm":
-        achieved = nbytes / decode_avg_s / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved = flops / decode_avg_s / 1e12
-        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    rl = roofline_of(nbytes, flops, decode_avg_s, peaks)
+    bound, achieved, peak, unit = rl["bound"], rl["achieved"], rl["peak"], rl["unit"]
+    step_p = percentiles(step_ms)
+    call_p = percentiles(decode_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -550,12 +671,20 @@ def run_cuda(args, rank, local, world):
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6.65 TB/s / 1.59 PFLOP/s"},
         "kernel_us": {"metadata": statistics.median(meta_ms) * 1e3,
-                      "decode_call": statistics.median(decode_ms) * 1e3,
-                      "step": statistics.median(step_ms) * 1e3},
+                      "decode_call": call_p[0] * 1e3, "decode_call_p10": call_p[1] * 1e3,
+                      "decode_call_p90": call_p[2] * 1e3,
+                      "step": step_p[0] * 1e3, "step_p10": step_p[1] * 1e3,
+                      "step_p90": step_p[2] * 1e3},
         "gpu_launches": ((5 + (s_q > 1)) if sparse_idx is not None else 3) * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": dict(clocks.summary(), window=(
+            "NVML samples every 5 ms from the first timed step to the end of the per-workload "
+            "sweep (graph replays of the same kernels); the timed region's own samples are in "
+            "clocks_timed_region")),
+        "clocks_timed_region": clocks.summary(0, timed_samples),
         "wall_s_timed_region": t_wall,
     }
+    if workloads is not None:
+        line["workloads"] = workloads
     if e2e is not None:
         line["e2e"] = e2e
     if append is not None:
@@ -686,6 +815,10 @@ def main():
                          "position (seeded uniform picks; bf16 cache)")
     ap.add_argument("--no-append", action="store_true",
                     help="skip timing the latent-cache append")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the sweep over every configuration")
+    ap.add_argument("--sweep-reps", type=int, default=100,
+                    help="graph replays per configuration in the sweep (each after an L2 flush)")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="approximate oracle time for the cpu_baseline sample")
     args = ap.parse_args()

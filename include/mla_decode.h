@@ -172,7 +172,9 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
  *
  * Limit: if mla_workspace_size(batch, s_q, h_q, dv, num_workers) exceeds
  * MLA_STATIC_SCRATCH_BYTES it returns MLA_ERR_SCRATCH_LIMIT and launches
- * nothing (fewer workers need less workspace).
+ * nothing (fewer workers need less workspace).  Null pointers, d / dv other
+ * than 576 / 512 and sizes below 1 are checked before the limit and reported
+ * as MLA_ERR_INVALID_ARG / MLA_ERR_UNSUPPORTED.
  * Every GPU that loads this part of the library holds the 48 MiB array until
  * the process exits.  All calls on a device share it and it keeps the last
  * call's contents (nothing in it needs to start at zero); calls that overlap

@@ -106,6 +106,51 @@ def _require(ok: bool, what: str):
         raise ValueError(f"invalid argument: {what}")
 
 
+def _shape(t: torch.Tensor, shape, dtype, what: str):
+    """t must be a contiguous `dtype` tensor of exactly `shape`."""
+    _require(t.dtype == dtype, f"{what} must be {dtype}")
+    _require(tuple(t.shape) == tuple(shape), f"{what} must have shape {tuple(shape)}, "
+             f"got {tuple(t.shape)}")
+    _require(t.is_contiguous(), f"{what} must be contiguous")
+
+
+def _check_decode_args(q, block_table, cache_seqlens, tile_md, num_splits, out, lse, workspace,
+                       device_status, dv, extra=()):
+    """Shapes, dtypes and devices of the decode's tensors.  The C ABI sees only
+    pointers, so a tensor of the wrong extent would be read or written past its
+    end on the device: every extent the kernels rely on is checked here."""
+    _require(q.dim() == 4 and q.shape[3] == D_QK, "q must be [batch, s_q, h_q, 576]")
+    b, s_q, h_q, _ = q.shape
+    _require(q.dtype == torch.bfloat16 and q.is_contiguous(), "q must be contiguous bf16")
+    _require(dv == D_V, "dv must be 512")
+    _require(block_table.dim() == 2 and block_table.shape[0] == b and block_table.shape[1] >= 1,
+             "block_table must be [batch, max_pages]")
+    _require(block_table.dtype == torch.int32 and block_table.is_contiguous(),
+             "block_table must be contiguous int32")
+    _shape(cache_seqlens, (b,), torch.int32, "cache_seqlens")
+    if tile_md is not None:
+        _require(tile_md.dim() == 2 and tile_md.shape[1] == MD_STRIDE and tile_md.shape[0] >= 1,
+                 "tile_md must be [num_workers, 8]")
+        _shape(tile_md, tuple(tile_md.shape), torch.int32, "tile_md")
+        _shape(num_splits, (b + 1,), torch.int32, "num_splits")
+    if out is not None:
+        _shape(out, (b, s_q, h_q, dv), torch.bfloat16, "out")
+    if lse is not None:
+        _shape(lse, (b, h_q, s_q), torch.float32, "lse")
+    if workspace is not None:
+        _require(workspace.dtype == torch.uint8 and workspace.dim() == 1 and
+                 workspace.is_contiguous(), "workspace must be a contiguous 1-D uint8 tensor")
+    if device_status is not None:
+        _require(device_status.dtype == torch.int32 and device_status.numel() >= 1 and
+                 device_status.is_contiguous(), "device_status must hold one int32")
+    dev = q.device
+    for t in (block_table, cache_seqlens, tile_md, num_splits, out, lse, workspace,
+              device_status, *extra):
+        if t is not None:
+            _require(t.device == dev, "every tensor must be on q's device")
+    return b, s_q, h_q
+
+
 def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
@@ -154,19 +199,15 @@ def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch
                        workspace: torch.Tensor | None = None,
                        device_status: torch.Tensor | None = None):
     """Paged MLA decode.  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q] fp32)."""
-    b, s_q, h_q, d = q.shape
+    b, s_q, h_q = _check_decode_args(q, block_table, cache_seqlens, tile_md, num_splits, out, lse,
+                                     workspace, device_status, dv, extra=(kcache,))
+    d = D_QK
     dev = q.device
-    for t in (q, kcache, block_table, cache_seqlens, tile_md, num_splits):
-        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
-                 "every tensor must be contiguous on q's CUDA device")
-    _require(q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16,
-             "q and kcache must be bf16")
-    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
-             "block_table and cache_seqlens must be int32")
+    _require(kcache.dtype == torch.bfloat16 and kcache.is_contiguous(),
+             "kcache must be contiguous bf16")
     _require(kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d,
              "kcache must be [num_blocks, 64, 576]")
-    _require(block_table.dim() == 2 and block_table.shape[0] == b,
-             "block_table must be [batch, max_pages]")
+    _require(q.is_cuda, "q must be on a CUDA device")
     num_workers = tile_md.shape[0]
     with torch.cuda.device(dev):
         if out is None:
@@ -274,19 +315,16 @@ def mla_decode_kvcache_fp8(q: torch.Tensor, kcache8: torch.Tensor, kscale: torch
                            device_status: torch.Tensor | None = None):
     """Paged MLA decode over an FP8 cache (codes kcache8 [nblk, 64, 576] uint8 and per-token
     scales kscale [nblk, 64] fp32).  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q])."""
-    b, s_q, h_q, d = q.shape
+    b, s_q, h_q = _check_decode_args(q, block_table, cache_seqlens, tile_md, num_splits, out, lse,
+                                     workspace, device_status, dv, extra=(kcache8, kscale))
+    d = D_QK
     dev = q.device
-    for t in (q, kcache8, kscale, block_table, cache_seqlens, tile_md, num_splits):
-        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
-                 "every tensor must be contiguous on q's CUDA device")
-    _require(q.dtype == torch.bfloat16 and kcache8.dtype == torch.uint8,
-             "q must be bf16 and kcache8 uint8")
-    _require(kscale.dtype == torch.float32 and tuple(kscale.shape) == tuple(kcache8.shape[:2]),
-             "kscale must be fp32 [num_blocks, 64]")
-    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
-             "block_table and cache_seqlens must be int32")
+    _require(kcache8.dtype == torch.uint8 and kcache8.is_contiguous(),
+             "kcache8 must be contiguous uint8")
     _require(kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == d,
              "kcache8 must be [num_blocks, 64, 576]")
+    _shape(kscale, tuple(kcache8.shape[:2]), torch.float32, "kscale")
+    _require(q.is_cuda, "q must be on a CUDA device")
     num_workers = tile_md.shape[0]
     with torch.cuda.device(dev):
         if out is None:
@@ -313,19 +351,19 @@ def mla_decode_sparse(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.
     """Sparse decode: each query position attends to the cached tokens listed in
     indices [b, s_q, topk] int32 (entries outside the sequence, or past the causal
     limit, are skipped).  Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q])."""
-    b, s_q, h_q, d = q.shape
+    b, s_q, h_q = _check_decode_args(q, block_table, cache_seqlens, None, None, out, lse,
+                                     workspace, device_status, dv, extra=(kcache, indices))
+    d = D_QK
     dev = q.device
-    for t in (q, kcache, block_table, cache_seqlens, indices):
-        _require(t.is_cuda and t.device == dev and t.is_contiguous(),
-                 "every tensor must be contiguous on q's CUDA device")
-    _require(q.dtype == torch.bfloat16 and kcache.dtype == torch.bfloat16,
-             "q and kcache must be bf16")
-    _require(block_table.dtype == torch.int32 and cache_seqlens.dtype == torch.int32,
-             "block_table and cache_seqlens must be int32")
-    _require(indices.dtype == torch.int32 and indices.dim() == 3,
-             "indices must be int32 [batch, s_q, topk]")
-    _require(indices.shape[0] == b and indices.shape[1] == s_q,
+    _require(kcache.dtype == torch.bfloat16 and kcache.is_contiguous(),
+             "kcache must be contiguous bf16")
+    _require(kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d,
+             "kcache must be [num_blocks, 64, 576]")
+    _require(indices.dtype == torch.int32 and indices.dim() == 3 and indices.is_contiguous(),
+             "indices must be contiguous int32 [batch, s_q, topk]")
+    _require(indices.shape[0] == b and indices.shape[1] == s_q and indices.shape[2] >= 1,
              "indices must be [batch, s_q, topk]")
+    _require(q.is_cuda, "q must be on a CUDA device")
     topk = indices.shape[2]
     with torch.cuda.device(dev):
         num_workers, _ = metadata_shape(b * s_q, h_q, 1)

@@ -12,7 +12,8 @@
 //   - The array is kStaticScratchBytes (48 MiB) per GPU.  Every GPU that loads
 //     this part of the library holds it until the process exits.
 //   - Calls whose workspace would exceed it are rejected with
-//     MLA_ERR_SCRATCH_LIMIT before anything is launched.
+//     MLA_ERR_SCRATCH_LIMIT before anything is launched (null pointers and bad
+//     sizes are reported as MLA_ERR_INVALID_ARG first).
 //   - All calls on a device share the one array, and it keeps whatever the
 //     last call left there.  The decode writes every partial it later reads, so
 //     nothing has to start at zero; but two calls that run on the GPU at the
@@ -65,7 +66,15 @@ int mla_decode_kvcache_static_scratch(const void* q, const void* kcache, int64_t
                                       const int32_t* tile_md, const int32_t* num_splits,
                                       int num_workers, void* out, float* lse,
                                       int32_t* device_status, void* stream) {
+  // The argument checks of mla_decode_kvcache that do not depend on the
+  // workspace come first, so that a call with a null pointer or a bad size
+  // reports MLA_ERR_INVALID_ARG whatever workspace its shape would need.
+  if (q == nullptr || kcache == nullptr || block_table == nullptr || cache_seqlens == nullptr ||
+      tile_md == nullptr || num_splits == nullptr || out == nullptr || lse == nullptr)
+    return MLA_ERR_INVALID_ARG;
   if (d != MLA_HEAD_DIM_QK || dv != MLA_HEAD_DIM_V) return MLA_ERR_UNSUPPORTED;
+  if (batch < 1 || s_q < 1 || h_q < 1 || bt_stride < 1 || num_workers < 1 || num_blocks < 1)
+    return MLA_ERR_INVALID_ARG;
   const size_t need = mla_workspace_size(batch, s_q, h_q, dv, num_workers);
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (need > kStaticScratchBytes) return MLA_ERR_SCRATCH_LIMIT;

@@ -230,3 +230,90 @@ def test_binding_rejects_bad_tensors_before_any_call():
                                   torch.zeros((1, 1), dtype=torch.int32),
                                   torch.ones(1, dtype=torch.int32),
                                   torch.zeros((1, 1, 4), dtype=torch.int32), 0.07)
+
+
+def _decode_args(b=2, s_q=1, h_q=16, nb=4, W=8):
+    import torch
+    return dict(
+        q=torch.zeros((b, s_q, h_q, 576), dtype=torch.bfloat16),
+        kcache=torch.zeros((nb, 64, 576), dtype=torch.bfloat16),
+        block_table=torch.zeros((b, 3), dtype=torch.int32),
+        cache_seqlens=torch.ones(b, dtype=torch.int32),
+        dv=512,
+        tile_md=torch.zeros((W, 8), dtype=torch.int32),
+        num_splits=torch.zeros(b + 1, dtype=torch.int32),
+        softmax_scale=0.07,
+        out=torch.zeros((b, s_q, h_q, 512), dtype=torch.bfloat16),
+        lse=torch.zeros((b, h_q, s_q), dtype=torch.float32),
+        workspace=torch.zeros(1 << 20, dtype=torch.uint8),
+        device_status=torch.zeros(1, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("field,bad,match", [
+    ("cache_seqlens", "short", "cache_seqlens must have shape"),
+    ("cache_seqlens", "int64", "cache_seqlens must be torch.int32"),
+    ("num_splits", "short", "num_splits must have shape"),
+    ("tile_md", "stride", r"tile_md must be \[num_workers, 8\]"),
+    ("tile_md", "int64", "tile_md must be torch.int32"),
+    ("out", "short", "out must have shape"),
+    ("out", "fp32", "out must be torch.bfloat16"),
+    ("lse", "transposed", "lse must have shape"),
+    ("lse", "fp16", "lse must be torch.float32"),
+    ("workspace", "fp32", "workspace must be a contiguous 1-D uint8"),
+    ("device_status", "int64", "device_status must hold one int32"),
+    ("block_table", "rows", r"block_table must be \[batch, max_pages\]"),
+    ("kcache", "page", r"kcache must be \[num_blocks, 64, 576\]"),
+    ("q", "dims", r"q must be \[batch, s_q, h_q, 576\]"),
+])
+def test_binding_checks_every_extent(field, bad, match):
+    # each tensor whose extent the kernels rely on is checked before the call;
+    # the C ABI itself sees only pointers
+    import torch
+    a = _decode_args()
+    t = a[field]
+    if bad == "short":
+        t = t.flatten()[:-1] if t.dim() == 1 else t[:-1]
+    elif bad == "int64":
+        t = t.to(torch.int64)
+    elif bad == "stride":
+        t = torch.zeros((t.shape[0], 4), dtype=torch.int32)
+    elif bad == "fp32":
+        t = t.float()
+    elif bad == "fp16":
+        t = t.half()
+    elif bad == "transposed":
+        t = t.transpose(1, 2).contiguous()
+    elif bad == "rows":
+        t = torch.zeros((1, 3), dtype=torch.int32)
+    elif bad == "page":
+        t = torch.zeros((4, 32, 576), dtype=torch.bfloat16)
+    elif bad == "dims":
+        t = torch.zeros((2, 1, 16, 512), dtype=torch.bfloat16)
+    a[field] = t
+    with pytest.raises(ValueError, match=match):
+        binding.mla_decode_kvcache(**a)
+
+
+def test_binding_well_formed_cpu_tensors_stop_at_device_check():
+    with pytest.raises(ValueError, match="CUDA device"):
+        binding.mla_decode_kvcache(**_decode_args())
+
+
+def test_static_scratch_checks_arguments_before_the_limit():
+    # a shape whose workspace exceeds the static array, but with a null pointer:
+    # the argument error is reported, not the limit
+    lib = binding.lib
+    b, s_q, h_q, nw = 1024, 1, 128, 74
+    assert binding.workspace_size(b, s_q, h_q, nw) > binding.STATIC_SCRATCH_BYTES
+    v = ctypes.c_void_p
+
+    def call(q=1 << 12, lse=1 << 12, d=576, batch=b):
+        return lib.mla_decode_kvcache_static_scratch(
+            v(q), v(1 << 12), 1, v(1 << 12), 1, v(1 << 12), batch, s_q, h_q, d, 512, 0.07, 0,
+            v(1 << 12), v(1 << 12), nw, v(1 << 12), v(lse), v(0), v(0))
+    assert call(q=0) == binding.MLA_ERR_INVALID_ARG
+    assert call(lse=0) == binding.MLA_ERR_INVALID_ARG
+    assert call(d=512) == binding.MLA_ERR_UNSUPPORTED
+    assert call(batch=0) == binding.MLA_ERR_INVALID_ARG
+    # well-formed arguments: the limit is reported, before any device call
+    assert call() == binding.MLA_ERR_SCRATCH_LIMIT

@@ -65,3 +65,18 @@ def test_reference_arm_under_torchrun_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_percentiles_and_roofline_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    med, p10, p90 = bench.percentiles(list(range(1, 102)))
+    assert (med, p10, p90) == (51, 11, 91)
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0}
+    # 1 GB in 2 ms at 1000 GB/s peak: HBM-bound, 500 GB/s achieved, half the peak
+    r = bench.roofline_of(1e9, 1e9, 2e-3, peaks)
+    assert r["bound"] == "hbm" and abs(r["achieved"] - 500.0) < 1e-9 and abs(r["frac"] - 0.5) < 1e-12
+    assert abs(r["bound_us"] - 1000.0) < 1e-6
+    # 1 TFLOP in 20 ms at 100 TFLOP/s: tensor-bound (10 ms against 1 ms of bytes)
+    r = bench.roofline_of(1e9, 1e12, 2e-2, peaks)
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.5) < 1e-12

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from mla_paged_latent_decode_b200 import synth
-from parity import (check_metadata, full_parity, run_cuda, sampled_parity, assert_close_out,
+from parity import (check_metadata, full_parity, full_size_parity, run_cuda, assert_close_out,
                     assert_close_lse, expected_workers)
 
 pytestmark = pytest.mark.gpu
@@ -132,11 +132,10 @@ def test_dominant_key_and_large_logits(cuda_device):
 
 
 @pytest.mark.parametrize("name", ["dsv3_decode", "varlen_h16", "spec_causal", "skewed_long"])
-def test_full_size_workloads_sampled(cuda_device, name):
+def test_full_size_workloads(cuda_device, name):
+    # every element of out and lse, in the launch configuration the benchmark times
     inp = synth.make_inputs(name, seed=0)
-    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
-    extra = [(0, 0, 0), (b - 1, s_q - 1, h_q - 1)]
-    sampled_parity(inp, cuda_device, n_rows=48, extra_rows=extra)
+    full_size_parity(inp, cuda_device)
 
 
 def test_default_workers_match_formula(cuda_device):

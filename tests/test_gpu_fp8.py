@@ -149,21 +149,18 @@ def test_fp8_decode_dominant_key(cuda_device):
     assert_close_lse(lse, ref_lse, "fp8 lse")
 
 
-def test_fp8_varlen_full_size_sampled(cuda_device):
+def test_fp8_varlen_full_size(cuda_device):
     # the memory-bound variable-length workload (128 sequences, 16 heads,
-    # lengths U[1, 8192]) in the default launch configuration
+    # lengths U[1, 8192]) in the default launch configuration; every element
     inp = synth.make_inputs("varlen_h16", seed=0)
     codes, scales = encode_cache(inp.kcache)
     out, lse, md, ns = run_fp8(inp, codes, scales, cuda_device)
     check_metadata(inp, dict(tile_md=md, num_splits=ns), md.shape[0])
     assert md.shape[0] == expected_workers(cuda_device, inp.s_q, inp.h_q)
-    g = np.random.default_rng(0)
-    rows = sorted({(int(g.integers(inp.batch)), 0, int(g.integers(inp.h_q))) for _ in range(48)})
-    ref_out, ref_lse = oracle.decode_rows(inp.q, dequantized(codes, scales), inp.block_table,
-                                          inp.cache_seqlens, inp.scale, False, rows)
-    assert_close_out(np.stack([out[i, j, h] for i, j, h in rows]), ref_out, "fp8 sampled out")
-    assert_close_lse(np.array([lse[i, h, j] for i, j, h in rows]), ref_lse, "fp8 sampled lse")
-    assert np.all(np.isfinite(out))
+    ref_out, ref_lse = oracle.decode(inp.q, dequantized(codes, scales), inp.block_table,
+                                     inp.cache_seqlens, inp.scale, False)
+    assert_close_out(out, ref_out, "fp8 out")
+    assert_close_lse(lse, ref_lse, "fp8 lse")
 
 
 def packed(codes, scales):

@@ -145,7 +145,7 @@ def test_more_workers_than_items(P):
 @pytest.mark.parametrize("W", [1, 2, 3, 5, 7])
 def test_brute_force_small(W, P):
     lengths = [0, 1, 63, 64, 65, 128, 129, 300]
-    for b in (1, 2, 3):
+    for b in (1, 2, 3, 4):
         for lens in itertools.product(lengths, repeat=b):
             check_plan(list(lens), W, P)
 

@@ -4,10 +4,12 @@ Some callers cannot call cudaMalloc (an engine that owns all device memory in
 its own arena, a loop that must never allocate or free), so they cannot hand
 mla_decode_kvcache a workspace for split partials.  The static-scratch entry
 point uses a fixed array inside the library instead.  These tests call it
-through the C ABI and check that it gives the same results as the ordinary
-entry point, within the decode's tolerance, on two calls in a row (the second
-call finds the first call's data still in the shared array), and that a
-workspace larger than the array is refused before anything runs.
+through the C ABI and check that it gives bit for bit the results of the
+ordinary entry point (both run the same kernels on the same split plan), and
+the oracle's within the decode's tolerance, over several calls in a row: each
+call finds the previous call's partials still in the shared array, including
+a call with more pieces than the one after it.  A workspace larger than the
+array is refused before anything runs.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -18,11 +20,11 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mla_paged_latent_decode_b200 import binding, synth
+from parity import assert_close_lse, assert_close_out
 
 pytestmark = pytest.mark.gpu
-
-OUT_ATOL, OUT_RTOL, LSE_ATOL = 1e-2, 1e-2, 1e-3
 
 
 def _p(t):
@@ -41,8 +43,12 @@ def test_static_scratch_matches_ordinary_entry_point(cuda_device):
     cases = [
         (synth.custom_workload(4, 2, 128, [700, 1, 3000, 64], causal=True), 20, 31),
         (synth.custom_workload(6, 1, 16, [5000, 90, 0, 4100, 64, 777]), 40, 32),
+        # many more pieces than the calls before and after it leave in the array
+        (synth.custom_workload(3, 1, 128, [2900, 4000, 1500]), 74, 33),
     ]
-    for w, num_workers, seed in cases:
+    # the first case again at the end: it reads an array that a call with more
+    # pieces has just filled
+    for w, num_workers, seed in cases + cases[:1]:
         inp = synth.make_inputs(w, seed=seed)
         q, kc = inp.q.to(cuda_device), inp.kcache.to(cuda_device)
         bt, sl = inp.block_table.to(cuda_device), inp.cache_seqlens.to(cuda_device)
@@ -57,12 +63,13 @@ def test_static_scratch_matches_ordinary_entry_point(cuda_device):
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert int(ns[-1].item()) > inp.batch, "the case must split sequences to use the scratch"
-        got, ref = out.float().cpu().numpy(), ref_out.float().cpu().numpy()
-        assert np.all(np.abs(got - ref) <= OUT_ATOL + OUT_RTOL * np.abs(ref))
-        gl, rl = lse.cpu().numpy(), ref_lse.cpu().numpy()
-        both_inf = np.isneginf(gl) & np.isneginf(rl)
-        with np.errstate(invalid="ignore"):
-            assert np.all(both_inf | (np.abs(gl - rl) <= LSE_ATOL))
+        # same kernels, same plan: the same bits
+        assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+        assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
+        want_out, want_lse = oracle.decode(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens,
+                                           inp.scale, inp.causal)
+        assert_close_out(out.float().cpu().numpy(), want_out, "static-scratch out")
+        assert_close_lse(lse.cpu().numpy(), want_lse, "static-scratch lse")
 
 
 def test_static_scratch_refuses_oversized_workspace(cuda_device):
