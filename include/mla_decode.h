@@ -353,6 +353,47 @@ int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
 /* mla_error_string -- static text for a status code (never NULL). */
 const char* mla_error_string(int status);
 
+/*
+ * mla_merge_partials -- merge decode results over disjoint parts of each
+ * sequence's cache by log-sum-exp: the exchange step of a decode whose cache is
+ * sharded across GPUs (each rank decodes the pages it holds, the ranks gather
+ * their results, and every rank merges them).
+ *
+ * The pages describe the cross-device form as partition-then-combine ("TPLA:
+ * Tensor Parallel Latent Attention...", abstract: attend per shard, then
+ * combine across devices).  Sharding the cached tokens keeps it exact:
+ *   lse = ln sum_r exp(lse_r),  out = sum_r exp(lse_r - lse) * out_r,
+ * with a part whose lse_r = -inf (no visible token there) weighing nothing, and
+ * out = 0, lse = -inf when every part is empty.
+ *
+ *   outs  [num_parts, batch, s_q, h_q, 512] bf16, device: part r's decode output
+ *         (normalised over part r's tokens), parts back to back.  16-B aligned.
+ *   lses  [num_parts, batch, h_q, s_q] fp32, device: part r's lse (natural log).
+ *   out   [batch, s_q, h_q, 512] bf16, device, 16-B aligned; lse [batch, h_q, s_q]
+ *         fp32, device.  May not overlap the inputs.
+ * The caller owns every buffer; nothing is allocated.  Asynchronous on `stream`.
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG (null, sizes < 1, more than 4096 parts,
+ * s_q * h_q > 65536, num_parts * batch * s_q * h_q >= 2^31, misalignment) or
+ * MLA_ERR_CUDA (launch failure).
+ */
+int mla_merge_partials(const void* outs, const float* lses, int num_parts, int batch, int s_q,
+                       int h_q, void* out, float* lse, void* stream);
+
+/*
+ * mla_set_wait_limit_ns -- limit of each bounded wait inside the decode kernels.
+ *
+ * Not part of the method (the pages have no counterpart): every wait of a
+ * decode kernel on a barrier gives up after this long, stops the CTA, lets the
+ * asynchronous copies and MMAs it has already issued finish, and reports
+ * MLA_ERR_DEVICE_TIMEOUT through device_status; nothing traps.  The default,
+ * 2 s, is far above any legitimate wait.  Lowering it makes the timeout path
+ * run on purpose, which is how the tests check it (a wait of a few microseconds
+ * cannot see its data arrive).  ns = 0 restores the default; values are
+ * clamped to [1000, 2e9].  Applies to decode calls launched after it, from any
+ * thread (a process-wide setting).  Returns the previous limit.
+ */
+uint64_t mla_set_wait_limit_ns(uint64_t ns);
+
 /* mla_version -- build identification string (never NULL). */
 const char* mla_version(void);
 

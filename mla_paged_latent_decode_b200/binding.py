@@ -32,7 +32,8 @@ STATIC_SCRATCH_BYTES = 48 << 20
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
            "mla_decode_kvcache_static_scratch", "mla_append_latent", "mla_release_pages",
            "mla_append_latent_fp8", "mla_decode_kvcache_fp8", "mla_sparse_workspace_size",
-           "mla_decode_sparse", "mla_error_string", "mla_version")
+           "mla_decode_sparse", "mla_merge_partials", "mla_set_wait_limit_ns",
+           "mla_error_string", "mla_version")
 
 
 class MLAError(RuntimeError):
@@ -78,6 +79,10 @@ def _load() -> ctypes.CDLL:
     lib.mla_release_pages.restype = i32
     lib.mla_error_string.argtypes = [i32]
     lib.mla_error_string.restype = ctypes.c_char_p
+    lib.mla_merge_partials.argtypes = [p, p, i32, i32, i32, i32, p, p, p]
+    lib.mla_merge_partials.restype = i32
+    lib.mla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.mla_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.mla_version.argtypes = []
     lib.mla_version.restype = ctypes.c_char_p
     return lib
@@ -93,6 +98,12 @@ def error_string(code: int) -> str:
 
 def version() -> str:
     return lib.mla_version().decode()
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Limit of each bounded wait inside the decode kernels (0 = the 2 s default).
+    Returns the previous limit."""
+    return int(lib.mla_set_wait_limit_ns(int(ns)))
 
 
 def _check(code: int, what: str):
@@ -122,7 +133,6 @@ def _check_decode_args(q, block_table, cache_seqlens, tile_md, num_splits, out, 
     _require(q.dim() == 4 and q.shape[3] == D_QK, "q must be [batch, s_q, h_q, 576]")
     b, s_q, h_q, _ = q.shape
     _require(q.dtype == torch.bfloat16 and q.is_contiguous(), "q must be contiguous bf16")
-    _require(dv == D_V, "dv must be 512")
     _require(block_table.dim() == 2 and block_table.shape[0] == b and block_table.shape[1] >= 1,
              "block_table must be [batch, max_pages]")
     _require(block_table.dtype == torch.int32 and block_table.is_contiguous(),
@@ -382,4 +392,32 @@ def mla_decode_sparse(q: torch.Tensor, kcache: torch.Tensor, block_table: torch.
             int(bool(causal)), num_workers, _ptr(workspace), workspace.numel(), _ptr(out),
             _ptr(lse), _ptr(device_status), _stream_handle(dev))
         _check(rc, "mla_decode_sparse")
+    return out, lse
+
+
+def merge_partials(outs: torch.Tensor, lses: torch.Tensor, out: torch.Tensor | None = None,
+                   lse: torch.Tensor | None = None):
+    """Merge decode results over disjoint parts of the cache by log-sum-exp.
+    outs [R, b, s_q, h_q, 512] bf16, lses [R, b, h_q, s_q] fp32 (one entry per part).
+    Returns (out [b, s_q, h_q, 512] bf16, lse [b, h_q, s_q] fp32)."""
+    _require(outs.dim() == 5 and outs.shape[4] == D_V, "outs must be [parts, b, s_q, h_q, 512]")
+    R, b, s_q, h_q, _ = outs.shape
+    _shape(outs, (R, b, s_q, h_q, D_V), torch.bfloat16, "outs")
+    _shape(lses, (R, b, h_q, s_q), torch.float32, "lses")
+    dev = outs.device
+    if out is not None:
+        _shape(out, (b, s_q, h_q, D_V), torch.bfloat16, "out")
+    if lse is not None:
+        _shape(lse, (b, h_q, s_q), torch.float32, "lse")
+    for t in (lses, out, lse):
+        if t is not None:
+            _require(t.device == dev, "every tensor must be on outs' device")
+    _require(outs.is_cuda, "outs must be on a CUDA device")
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+        _check(lib.mla_merge_partials(_ptr(outs), _ptr(lses), R, b, s_q, h_q, _ptr(out), _ptr(lse),
+                                      _stream_handle(dev)), "mla_merge_partials")
     return out, lse

@@ -16,6 +16,8 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
+// Limit of each bounded wait inside the decode kernels (mla_set_wait_limit_ns).
+std::atomic<uint64_t> g_wait_ns{mla::kWaitLimitNs};
 
 int current_sm_count(int* sms) {
   int dev = 0;
@@ -179,6 +181,29 @@ const char* mla_error_string(int status) {
   }
 }
 
+int mla_merge_partials(const void* outs, const float* lses, int num_parts, int batch, int s_q,
+                       int h_q, void* out, float* lse, void* stream) {
+  if (outs == nullptr || lses == nullptr || out == nullptr || lse == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (num_parts < 1 || num_parts > 4096 || batch < 1 || s_q < 1 || h_q < 1)
+    return MLA_ERR_INVALID_ARG;
+  const int64_t nrows = static_cast<int64_t>(batch) * s_q * h_q;
+  if (static_cast<int64_t>(s_q) * h_q > 65536 || nrows * num_parts >= (int64_t(1) << 31))
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(outs, 16) || !aligned(out, 16) || !aligned(lses, 4) || !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  cudaError_t e = mla::launch_merge(outs, lses, num_parts, nrows, s_q, h_q, out, lse,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+uint64_t mla_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) ns = mla::kWaitLimitNs;
+  if (ns < 1000) ns = 1000;
+  if (ns > mla::kWaitLimitNs) ns = mla::kWaitLimitNs;
+  return g_wait_ns.exchange(ns);
+}
+
 const char* mla_version(void) {
   return "mla_paged_latent_decode_b200 sm_100a (tcgen05 pair decode for >64 query rows, M=64 decode otherwise)";
 }
@@ -269,18 +294,19 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   p.rows = rows;
   p.causal = causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (uses_pairs(s_q, h_q)) {
-    // K part: 32 token rows x 3 chunks per box; V part: 64 rows x 2 chunks
-    CUtensorMap tm_kpart, tm_vpart;
-    if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, 3)) return MLA_ERR_CUDA;
-    if (!make_chunk_map(&tm_vpart, kcache, cache_rows, 64, 2)) return MLA_ERR_CUDA;
+    // K part: 32 token rows x all 9 chunks per box; peer-token values: 32 rows x 4 chunks
+    CUtensorMap tm_kpart, tm_vx;
+    if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, mla::kDqk / 64)) return MLA_ERR_CUDA;
+    if (!make_chunk_map(&tm_vx, kcache, cache_rows, 32, 4)) return MLA_ERR_CUDA;
     CUtensorMap tm_po, tm_out;
     if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
     if (!make_out_map(&tm_out, out, static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)))
       return MLA_ERR_CUDA;
-    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vpart, tm_po, tm_out, p, num_workers, st) !=
+    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vx, tm_po, tm_out, p, num_workers, st) !=
         cudaSuccess)
       return MLA_ERR_CUDA;
   } else {
@@ -346,6 +372,7 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   p.rows = rows;
   p.causal = causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mla::launch_decode_fp8(tm_q, tm_page8, p, num_workers, st) != cudaSuccess)
     return MLA_ERR_CUDA;

@@ -12,12 +12,23 @@
 //                  (all 576 dims) as its half of B; each CTA receives S for its
 //                  64 rows and all 64 tokens.  Dims 0..383 of Q are read from
 //                  tensor memory, dims 384..575 from shared memory.
-//   O += P . V     N = 256 dv per MMA, two MMAs: CTA r supplies, for all 64
-//                  tokens, dv 256h+128r .. 256h+128r+127 of MMA h as its half of B.
-// So each CTA loads its 32 token rows in full (K part, 36 KB) and its 256
-// columns of dv for all 64 tokens (V part, 32 KB); the two CTAs together read
-// each page from HBM once.  Both parts are TMA boxes through the block table,
-// with 128-byte swizzle; their completion is counted on the leader's barriers.
+//   O += P . V     N = 256 dv per MMA, two MMAs: CTA 0 supplies dv 128h..128h+127
+//                  of MMA h and CTA 1 dv 256+128h..256+128h+127, for all 64 tokens.
+// Each CTA loads its 32 token rows in full (K part, 36 KB, nine 64-dim chunks of
+// 32 rows x 128 bytes) into a ring slot.  The same slot then serves as V:
+//   PV K-steps 0-1 (tokens  0..31) read chunks 0..3 of the slot,
+//   PV K-steps 2-3 (tokens 32..63) read chunks 4..7,
+// at the same shared-memory offsets in both CTAs (a pair MMA has one descriptor).
+// CTA 0's chunks 0..3 already hold what it supplies for tokens 0..31 (its own
+// tokens, dims 0..255), and CTA 1's chunks 4..7 what it supplies for tokens
+// 32..63.  The other half is the peer's tokens: once the QK^T MMAs have read
+// them, CTA 0 overwrites its chunks 4..7 with tokens 32..63 x dims 0..255 and
+// CTA 1 its chunks 0..3 with tokens 0..31 x dims 256..511 (16 KB each, one TMA
+// box; the bytes were just read from HBM by the peer, so they come from L2).
+// Shared memory therefore receives 1.44x the page bytes (36 + 16 KB per CTA
+// for a 72 KB page), and HBM is read once.  Both loads are TMA boxes through
+// the block table with 128-byte swizzle; their completion is counted on the
+// leader's barriers.
 //
 // Tensor memory per CTA (512 columns, all 128 lanes):
 //   O   columns   0..255  64 rows x 512 fp32: lane L holds row L % 64, dv half
@@ -27,7 +38,8 @@
 //   Q   columns 320..511  dims 0..383 of the 64 rows, two bf16 per column, each
 //                         row held in lanes L and L + 64
 // The rest of Q (dims 384..575, 24 KB) stays in shared memory, which leaves room
-// for three K-part slots, two V-part slots and two P buffers.
+// for five 36 KB slots and two P buffers.  A slot is held from its K-part load
+// until PV of its page has completed.
 //
 // The K-part ring also stages the query rows: per piece, two ring entries carry
 // dims 0..255 and 256..383 of this CTA's 64 rows (plain TMA, counted on this
@@ -39,7 +51,8 @@
 //              of row L % 64; the two halves of a row exchange maxima and sums
 //              through shared memory.
 //   warp 4     TMA: query rows and K parts (both CTAs).
-//   warp 8     TMA: V parts (both CTAs).
+//   warp 8     TMA: the peer-token value chunks (both CTAs), each as soon as the
+//              QK^T MMAs have read the chunks it replaces.
 //   warps 5, 7 QK^T of even / odd pages (leader CTA only); warp 5 also
 //              allocates the pair's tensor memory in each CTA.
 //   warp 6     PV (leader CTA only).
@@ -50,6 +63,8 @@
 // Efficient Decoding...", sections 4.2.1-4.2.3: TMA prefetch of 64-row latent
 // blocks, tensor cores for QK^T and PV, softmax fused in the kernel), mapped
 // onto the pair tensor-core instructions of sm_100a.
+#include <atomic>
+
 #include "mla_kernels.cuh"
 #include "sm100_ptx.cuh"
 
@@ -72,44 +87,43 @@ constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // dims 384..575 stay in 
 constexpr int kQStageA = 4;               // first staging entry: chunks 0..3
 constexpr int kQ2Bytes = kQSmemChunks * kChunk;        // 24576
 constexpr int kKBytes = kChunks * kHalfChunk;          // 36864: 32 tokens x 576
-constexpr int kVBytes = 4 * kChunk;                    // 32768: 64 tokens x 256 dv
+constexpr int kXChunks = 4;                            // chunks replaced by peer-token values
+constexpr int kXBytes = kXChunks * kHalfChunk;         // 16384: 32 tokens x 256 dv
 constexpr int kPBytes = kChunk;                        // 64 rows x 64 tokens
-constexpr int kKSlots = 3;
-constexpr int kVSlots = 2;
-// A K-part slot is handed back in three groups of three 64-dim chunks, each as
-// soon as the QK^T MMAs reading it have completed, so the producer refills the
-// start of a slot while the end is still being read.
-constexpr int kKGroups = 3;
-constexpr int kChunksPerGroup = 3;
-constexpr int kKStepsPerGroup = kChunksPerGroup * 4;
+constexpr int kKSlots = 5;
 constexpr int kQKSteps = kDqk / 16;                    // 36
 constexpr int kQTmemKSteps = kQTmemChunks * 4;         // 24
-static_assert(kKGroups * kChunksPerGroup == kChunks, "K-part groups cover the page");
+// QK^T K-steps after which chunks 0..3 (resp. 4..7) of the slot have been issued
+constexpr int kXDoneStep0 = 4 * kXChunks - 1;          // 15
+constexpr int kXDoneStep1 = 8 * kXChunks - 1;          // 31
 static_assert(kQStageA * kChunk <= kKBytes && (kQTmemChunks - kQStageA) * kChunk <= kKBytes,
               "query staging entries fit a K-part slot");
 
 constexpr int kOffQ2 = 0;
 constexpr int kOffK = kOffQ2 + kQ2Bytes;
-constexpr int kOffV = kOffK + kKSlots * kKBytes;
-constexpr int kOffP = kOffV + kVSlots * kVBytes;
+constexpr int kOffP = kOffK + kKSlots * kKBytes;
 constexpr int kOffX = kOffP + 2 * kPBytes;       // row-half exchange: [2 pages][2 halves][64] f32
 constexpr int kOffL = kOffX + 2 * 2 * 64 * 4;    // epilogue sum exchange: [2 pieces][2 halves][64] f32
 constexpr int kOffBar = kOffL + 2 * 2 * 64 * 4;
-static_assert(kOffK % 1024 == 0 && kKBytes % 1024 == 0 && kOffV % 1024 == 0 &&
-                  kOffP % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
+static_assert(kOffK % 1024 == 0 && kKBytes % 1024 == 0 && kOffP % 1024 == 0,
+              "swizzled tiles start on 1024-byte boundaries");
 enum Bar {
-  kKFull0 = 0,                                    // leader: K parts of both CTAs
-  kVFull0 = kKFull0 + kKSlots,                    // leader: V parts of both CTAs
-  kQFull = kVFull0 + kVSlots,                     // leader: Q dims 384..575 of both CTAs
-  kKEmpty0,                                       // both: pair commits (multicast),
-                                                  //   [slot][chunk group]
-  kVEmpty0 = kKEmpty0 + kKSlots * kKGroups,
-  kQEmpty = kVEmpty0 + kVSlots,
+  kKFull0 = 0,                                    // leader: K parts of both CTAs, per slot
+  kVFull0 = kKFull0 + kKSlots,                    // leader: peer-token values of both CTAs
+  kQFull = kVFull0 + kKSlots,                     // leader: Q dims 384..575 of both CTAs
+  kKEmpty0,                                       // both: pair commits (multicast), per slot:
+                                                  //   PV of the slot's page (or the query
+                                                  //   copies of a staging entry) is done
+  kXFree0 = kKEmpty0 + kKSlots,                   // both: pair commits, [slot][2]: QK^T has
+                                                  //   read chunks 0..3 / 4..7 of the slot
+  kQEmpty = kXFree0 + 2 * kKSlots,
   kSFull0, kSFull1, kPvDone0, kPvDone1, kOFull,   // both: pair commits (multicast)
   kSFree0, kSFree1, kPFull0, kPFull1, kQReady,    // leader: softmax warps of both CTAs
   kQStage,                                        // local: this CTA's query staging copies
   kXBar, kLBar,                                   // local: softmax exchanges
-  kNumBars
+  kDrain0,                                        // leader: MMA drain after an abort, one
+                                                  //   per issuing warp (5, 6, 7)
+  kNumBars = kDrain0 + 3
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffMisc + 16;
@@ -153,8 +167,8 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
 }
 
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
-  const bool ok = mbar_wait_cluster(bar, parity, abort, kWaitLimitNs);
+                                                  volatile int* abort, uint64_t limit_ns) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -177,13 +191,13 @@ __device__ __forceinline__ void warp_arrive_leader(uint64_t* bar, uint32_t rank,
 __device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar,
                                                 volatile int* abort_flag, uint32_t tmem_q, int r,
                                                 uint32_t rank, int lane, int& entries,
-                                                int& qcopies) {
+                                                int& qcopies, uint64_t wait_ns) {
   const uint8_t* qa = sk + (entries % kKSlots) * kKBytes;
   const uint8_t* qb = sk + ((entries + 1) % kKSlots) * kKBytes;
   entries += 2;
-  if (qcopies > 0 && !warp_wait_cluster(&bar[kQEmpty], (qcopies - 1) & 1, abort_flag))
+  if (qcopies > 0 && !warp_wait_cluster(&bar[kQEmpty], (qcopies - 1) & 1, abort_flag, wait_ns))
     return false;
-  if (!warp_wait_cluster(&bar[kQStage], qcopies & 1, abort_flag)) return false;
+  if (!warp_wait_cluster(&bar[kQStage], qcopies & 1, abort_flag, wait_ns)) return false;
   ++qcopies;
   for (int c = 0; c < kQTmemChunks; ++c) {
     const uint8_t* rowp = (c < kQStageA ? qa + c * kChunk : qb + (c - kQStageA) * kChunk) + r * 128;
@@ -207,7 +221,7 @@ __device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kpart,
-                       const __grid_constant__ CUtensorMap tm_vpart,
+                       const __grid_constant__ CUtensorMap tm_vx,
                        const __grid_constant__ CUtensorMap tm_po,
                        const __grid_constant__ CUtensorMap tm_out, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -215,7 +229,6 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sq2 = smem + kOffQ2;
   uint8_t* sk = smem + kOffK;
-  uint8_t* sv = smem + kOffV;
   uint8_t* sp = smem + kOffP;
   float* sx = reinterpret_cast<float*>(smem + kOffX);
   float* sl = reinterpret_cast<float*>(smem + kOffL);
@@ -237,15 +250,15 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     return;
   }
   const int row0 = rb2 * 128 + 64 * static_cast<int>(rank);  // first query row of this CTA
+  const uint64_t wait_ns = p.wait_ns;  // limit of every bounded wait (normally kWaitLimitNs)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&bar[kKFull0 + s], 1);
-      for (int grp = 0; grp < kKGroups; ++grp) mbar_init(&bar[kKEmpty0 + s * kKGroups + grp], 1);
-    }
-    for (int s = 0; s < kVSlots; ++s) {
       mbar_init(&bar[kVFull0 + s], 1);
-      mbar_init(&bar[kVEmpty0 + s], 1);
+      mbar_init(&bar[kKEmpty0 + s], 1);
+      mbar_init(&bar[kXFree0 + 2 * s], 1);
+      mbar_init(&bar[kXFree0 + 2 * s + 1], 1);
     }
     mbar_init(&bar[kQFull], 1);
     mbar_init(&bar[kQEmpty], 2);  // one commit from each QK^T warp
@@ -262,6 +275,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar[kQStage], 1);
     mbar_init(&bar[kXBar], 32 * kSoftmaxWarps);
     mbar_init(&bar[kLBar], 32 * kSoftmaxWarps);
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[kDrain0 + i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -292,7 +306,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int qrow = pz.seq * p.rows + row0;
         // dims 384..575 of the query rows: shared memory, counted on the leader
         if (qloads > 0) {
-          ok = mbar_wait_cluster(&bar[kQEmpty], (qloads - 1) & 1, abort_flag, kWaitLimitNs);
+          ok = mbar_wait_cluster(&bar[kQEmpty], (qloads - 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
         }
         if (rank == 0) mbar_arrive_expect_tx(&bar[kQFull], 2 * kQ2Bytes);
@@ -302,9 +316,9 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         // dims 0..383: two staging entries of the K ring, counted on this CTA's barrier
         for (int e = 0; e < 2; ++e) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
-          for (int grp = 0; grp < kKGroups && use > 0 && ok; ++grp)
-            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot * kKGroups + grp], (use - 1) & 1,
-                                   abort_flag, kWaitLimitNs);
+          if (use > 0)
+            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
+                                   wait_ns);
           if (!ok) break;
           if (e == 0) mbar_arrive_expect_tx(&bar[kQStage], kQTmemChunks * kChunk);
           uint8_t* dst = sk + slot * kKBytes;
@@ -320,49 +334,50 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int j = 0; j < pz.npg && ok; ++j, ++entries) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
           const int page = __ldg(bt + pz.pg0 + j);
-          uint8_t* dst = sk + slot * kKBytes;
-          for (int grp = 0; grp < kKGroups; ++grp) {
-            if (use > 0) {
-              ok = mbar_wait_cluster(&bar[kKEmpty0 + slot * kKGroups + grp], (use - 1) & 1,
-                                     abort_flag, kWaitLimitNs);
-              if (!ok) break;
-            }
-            // group 0 released means the QK^T warp has consumed the slot's previous
-            // fill, so the leader's full barrier is in the phase of this entry
-            if (grp == 0 && rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
-            // one box: 32 token rows x the group's 3 chunks
-            tma_load_3d_pair(dst + grp * kChunksPerGroup * kHalfChunk, &tm_kpart, 0,
-                             page * kPage + 32 * static_cast<int>(rank), grp * kChunksPerGroup,
-                             &bar[kKFull0 + slot]);
+          if (use > 0) {
+            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
+                                   wait_ns);
+            if (!ok) break;
           }
+          // the slot's previous entry is consumed, so the leader's full barrier is
+          // in the phase of this entry
+          if (rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
+          // one box: this CTA's 32 token rows x all nine chunks
+          tma_load_3d_pair(sk + slot * kKBytes, &tm_kpart, 0,
+                           page * kPage + 32 * static_cast<int>(rank), 0, &bar[kKFull0 + slot]);
         }
       }
     }
   } else if (warp == kTmaVWarp) {
-    // ------------------------------------------------------------ V parts
+    // ------------------------------------------------------------ peer-token values
+    // CTA 0 replaces chunks 4..7 of each page's slot with tokens 32..63 x dims
+    // 0..255, CTA 1 chunks 0..3 with tokens 0..31 x dims 256..511, each once the
+    // QK^T MMAs have read the chunks being replaced (of both CTAs: one commit).
     if (lane == 0) {
-      prefetch_tensormap(&tm_vpart);
-      int pages = 0;
+      prefetch_tensormap(&tm_vx);
+      const int xgrp = rank == 0 ? 1 : 0;
+      const int dst_chunk = rank == 0 ? kXChunks : 0;
+      const int src_row = rank == 0 ? 32 : 0, src_chunk = rank == 0 ? 0 : kXChunks;
+      int entries = 0;
+      uint32_t xbits = 0;  // parity of the next phase of each slot's X-free barrier
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (pz.npg == 0) continue;
+        entries += 2;  // the piece's query staging entries
         const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
-        for (int j = 0; j < pz.npg; ++j, ++pages) {
-          const int slot = pages % kVSlots, use = pages / kVSlots;
-          if (use > 0) {
-            ok = mbar_wait_cluster(&bar[kVEmpty0 + slot], (use - 1) & 1, abort_flag,
-                                   kWaitLimitNs);
-            if (!ok) break;
-          }
+        for (int j = 0; j < pz.npg; ++j, ++entries) {
+          const int slot = entries % kKSlots;
           const int page = __ldg(bt + pz.pg0 + j);
-          if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kVBytes);
-          uint8_t* dst = sv + slot * kVBytes;
-          // sub-chunks 2h, 2h + 1 hold dv blocks 4h + 2 rank, +1 (64 dv each): one box
-          // of 64 rows x 2 chunks per h
-          for (int h = 0; h < 2; ++h)
-            tma_load_3d_pair(dst + 2 * h * kChunk, &tm_vpart, 0, page * kPage,
-                             4 * h + 2 * static_cast<int>(rank), &bar[kVFull0 + slot]);
+          ok = mbar_wait_cluster(&bar[kXFree0 + 2 * slot + xgrp], (xbits >> slot) & 1u, abort_flag,
+                                 wait_ns);
+          if (!ok) break;
+          xbits ^= 1u << slot;
+          // the PV of the slot's previous page is done (its K part was reloaded
+          // after it), so the leader's V barrier is in the phase of this page
+          if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kXBytes);
+          tma_load_3d_pair(sk + slot * kKBytes + dst_chunk * kHalfChunk, &tm_vx, 0,
+                           page * kPage + src_row, src_chunk, &bar[kVFull0 + slot]);
         }
       }
     }
@@ -380,28 +395,26 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (pz.npg == 0) continue;
         const int stage_a = entries % kKSlots, stage_b = (entries + 1) % kKSlots;
         entries += 2;
-        ok = mbar_wait_cluster(&bar[kQFull], qloads & 1, abort_flag, kWaitLimitNs) &&
-             mbar_wait_cluster(&bar[kQReady], qloads & 1, abort_flag, kWaitLimitNs);
+        ok = mbar_wait_cluster(&bar[kQFull], qloads & 1, abort_flag, wait_ns) &&
+             mbar_wait_cluster(&bar[kQReady], qloads & 1, abort_flag, wait_ns);
         ++qloads;
         if (!ok) break;
         tc_fence_after();
         if (parity == 0) {  // both CTAs hold Q in tensor memory: the staging slots are free
-          for (int grp = 0; grp < kKGroups; ++grp) {
-            umma_commit_pair(&bar[kKEmpty0 + stage_a * kKGroups + grp]);
-            umma_commit_pair(&bar[kKEmpty0 + stage_b * kKGroups + grp]);
-          }
+          umma_commit_pair(&bar[kKEmpty0 + stage_a]);
+          umma_commit_pair(&bar[kKEmpty0 + stage_b]);
         }
         for (int j = 0; j < pz.npg && ok; ++j) {
           const int g = pages + j, b = g & 1, entry = entries + j;
           if (b != parity) continue;
           if (g >= 2) {  // both CTAs' softmax have read S of page g - 2 from buffer b
             ok = mbar_wait_cluster(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag,
-                                   kWaitLimitNs);
+                                   wait_ns);
             if (!ok) break;
           }
           const int slot = entry % kKSlots;
           ok = mbar_wait_cluster(&bar[kKFull0 + slot], (entry / kKSlots) & 1, abort_flag,
-                                 kWaitLimitNs);
+                                 wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint64_t b0 = smem_desc_sw128(k_base + slot * kKBytes, 16, 1024);
@@ -418,11 +431,11 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
               const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
               umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
             }
-            if (kk % kKStepsPerGroup == kKStepsPerGroup - 1 && kk != kQKSteps - 1)
-              umma_commit_pair(&bar[kKEmpty0 + slot * kKGroups + kk / kKStepsPerGroup]);
+            // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
+            if (kk == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
+            if (kk == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
           }
           umma_commit_pair(&bar[kSFull0 + b]);
-          umma_commit_pair(&bar[kKEmpty0 + slot * kKGroups + kKGroups - 1]);
         }
         if (!ok) break;
         umma_commit_pair(&bar[kQEmpty]);  // this warp's reads of Q for the piece are done
@@ -433,32 +446,41 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------ PV issuer (leader)
     if (rank == 0 && lane == 0) {
-      int pages = 0;
+      int pages = 0, entries = 0;
+      uint32_t vbits = 0;  // parity of the next phase of each slot's V barrier
       bool ok = true;
-      const uint32_t v_base = smem_addr(sv), p_base = smem_addr(sp);
+      const uint32_t k_base = smem_addr(sk), p_base = smem_addr(sp);
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (pz.npg == 0) continue;
-        for (int j = 0; j < pz.npg; ++j) {
-          const int g = pages + j, slot = g % kVSlots, pb = g & 1;
-          ok = mbar_wait_cluster(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, kWaitLimitNs);
+        entries += 2;  // the piece's query staging entries
+        for (int j = 0; j < pz.npg; ++j, ++entries) {
+          const int g = pages + j, slot = entries % kKSlots, pb = g & 1;
+          ok = mbar_wait_cluster(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
-          ok = mbar_wait_cluster(&bar[kVFull0 + slot], (g / kVSlots) & 1, abort_flag,
-                                 kWaitLimitNs);
+          ok = mbar_wait_cluster(&bar[kVFull0 + slot], (vbits >> slot) & 1u, abort_flag,
+                                 wait_ns);
           if (!ok) break;
+          vbits ^= 1u << slot;
           tc_fence_after();
-          const uint32_t vt = v_base + slot * kVBytes;
+          const uint32_t st = k_base + slot * kKBytes;
           const uint32_t pt = p_base + pb * kPBytes;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int kk = 0; kk < kPage / 16; ++kk) {
+              // tokens 16kk..16kk+15: chunk block 0..3 (tokens 0..31) or 4..7
+              // (tokens 32..63) of the slot, 16 rows of 128 bytes per K-step;
+              // this CTA's 128 dv of MMA h are chunks 2h, 2h + 1 of the block
+              // (LBO = one 32-row chunk, SBO = 8 rows)
+              const uint32_t vaddr = st + ((kk >> 1) * kXChunks + 2 * h) * kHalfChunk +
+                                     (kk & 1) * 2048;
               umma_bf16_ss_pair(tmem + kTmemO + 128 * h, smem_desc_sw128(pt + kk * 32, 16, 1024),
-                                smem_desc_sw128(vt + 2 * h * kChunk + kk * 2048, kChunk, 1024),
-                                kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                                smem_desc_sw128(vaddr, kHalfChunk, 1024), kIdescPV,
+                                (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          umma_commit_pair(&bar[kVEmpty0 + slot]);
+          umma_commit_pair(&bar[kKEmpty0 + slot]);
           umma_commit_pair(&bar[kPvDone0 + pb]);
         }
         if (!ok) break;
@@ -493,13 +515,13 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (pz.npg > 0) {
         if (!q_copied_ahead) {
           ok = copy_query_rows(sk, bar, abort_flag, tmem + quarter + kTmemQ, r, rank, lane, entries,
-                               qcopies);
+                               qcopies, wait_ns);
           if (!ok) break;
         }
         q_copied_ahead = false;
         for (int j = 0; j < pz.npg; ++j) {
           const int g = pages + j, pb = g & 1;
-          ok = warp_wait_cluster(&bar[kSFull0 + pb], (g >> 1) & 1, abort_flag);
+          ok = warp_wait_cluster(&bar[kSFull0 + pb], (g >> 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
           tc_fence_after();
           uint32_t s[32];
@@ -519,7 +541,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           float* xb = sx + pb * 128;
           xb[th * 64 + r] = mx;
           mbar_arrive(&bar[kXBar]);
-          ok = warp_wait_cluster(&bar[kXBar], g & 1, abort_flag);
+          ok = warp_wait_cluster(&bar[kXBar], g & 1, abort_flag, wait_ns);
           if (!ok) break;
           mx = fmaxf(mx, xb[(th ^ 1) * 64 + r]);
           float alpha = 1.f;
@@ -541,7 +563,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           // PV of a piece overwrites O, so its page needs no rescale.
           if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
             ok = warp_wait_cluster(&bar[kPvDone0 + ((g - 1) & 1)], ((g - 1) >> 1) & 1,
-                                   abort_flag);
+                                   abort_flag, wait_ns);
             if (!ok) break;
             tc_fence_after();
             for (int cb = 0; cb < 256; cb += 16) {
@@ -556,7 +578,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
           // P buffer pb was last read by PV of page g - 2
           if (g >= 2) {
-            ok = warp_wait_cluster(&bar[kPvDone0 + pb], ((g >> 1) - 1) & 1, abort_flag);
+            ok = warp_wait_cluster(&bar[kPvDone0 + pb], ((g >> 1) - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
           }
           // P row r, tokens 32 th .. 32 th + 31: 16-byte units 4 th .. 4 th + 3 (swizzled)
@@ -572,7 +594,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           warp_arrive_leader(&bar[kPFull0 + pb], rank, lane);
         }
         if (!ok) break;
-        ok = warp_wait_cluster(&bar[kOFull], pieces_done & 1, abort_flag);
+        ok = warp_wait_cluster(&bar[kOFull], pieces_done & 1, abort_flag, wait_ns);
         ++pieces_done;
         entries += pz.npg;
         pages += pz.npg;
@@ -583,7 +605,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int pn = pc + 1; pn < npieces; ++pn) {
           if (piece_of(md, pn, p.seqlens, p.bt_stride).npg > 0) {
             ok = copy_query_rows(sk, bar, abort_flag, tmem + quarter + kTmemQ, r, rank, lane,
-                                 entries, qcopies);
+                                 entries, qcopies, wait_ns);
             q_copied_ahead = true;
             break;
           }
@@ -601,7 +623,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       float* lb = sl + (pc & 1) * 128;
       lb[th * 64 + r] = l;
       mbar_arrive(&bar[kLBar]);
-      ok = warp_wait_cluster(&bar[kLBar], pc & 1, abort_flag);
+      ok = warp_wait_cluster(&bar[kLBar], pc & 1, abort_flag, wait_ns);
       if (!ok) break;
       const float lt = l + lb[(th ^ 1) * 64 + r];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
@@ -614,7 +636,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         // earlier, TMA stores would queue with the next piece's page loads.
         for (int h = 0; h < 2; ++h) {
           for (int cb = 0; cb < 128; cb += 64) {
-            const int col = 256 * h + 128 * th + cb;
+            const int col = 128 * h + 256 * th + cb;
             uint32_t w[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -653,7 +675,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int64_t orow0 = static_cast<int64_t>(pz.seq) * p.rows + wrow0;
         for (int h = 0; h < 2; ++h) {
           for (int cb = 0; cb < 128; cb += 32) {
-            const int col = 256 * h + 128 * th + cb;
+            const int col = 128 * h + 256 * th + cb;
             uint32_t o[32];
             if (pz.npg > 0) {
               tmem_ld32(tmem + quarter + kTmemO + 128 * h + cb, o);
@@ -721,6 +743,19 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 
   if (warp < kSoftmaxWarps && lane == 0) tma_store_wait_all();  // partial outputs written
+  // After an abort, work this CTA issued may still be in flight: pair MMAs of the
+  // leader's issuing threads (each waits for its own to complete, through a
+  // commit), and TMA loads of either CTA (they cannot be cancelled and land
+  // within microseconds; a grace period covers them).  Both must be done before
+  // the shared and tensor memory they write is released at the exit.
+  if (*abort_flag) {
+    if (rank == 0 && lane == 0 && warp >= kQkEvenWarp && warp <= kQkOddWarp) {
+      uint64_t* db = &bar[kDrain0 + (warp - kQkEvenWarp)];
+      umma_commit_leader(db);
+      mbar_wait_drain(db, 0, kWaitLimitNs);
+    }
+    if (threadIdx.x == 0) abort_grace();
+  }
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no pair MMA still writes either CTA's tensor memory
@@ -734,19 +769,19 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 }  // namespace
 
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
-                               const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
+                               const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
                                const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
                                cudaStream_t stream) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // per device: attribute set
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (!configured[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   const int blocks128 = (p.rows + 127) / 128;
   cudaLaunchConfig_t cfg = {};
@@ -763,20 +798,21 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vpart, tm_po, tm_out, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vx, tm_po, tm_out, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // Pairs (clusters of 2) of this kernel that fit on the device at once.
 cudaError_t pair_kernel_max_clusters(int* clusters) {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64];  // per device: 0 until computed
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (cached[dev] > 0) {
-    *clusters = cached[dev];
+  const int known = cached[dev].load(std::memory_order_acquire);
+  if (known > 0) {
+    *clusters = known;
     return cudaSuccess;
   }
   e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -797,7 +833,7 @@ cudaError_t pair_kernel_max_clusters(int* clusters) {
   e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel, &cfg);
   if (e != cudaSuccess) return e;
   if (n < 1) n = 1;
-  cached[dev] = n;
+  cached[dev].store(n, std::memory_order_release);
   *clusters = n;
   return cudaSuccess;
 }

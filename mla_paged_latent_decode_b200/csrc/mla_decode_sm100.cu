@@ -87,7 +87,8 @@ struct Cfg {
   static constexpr int kSFree0 = kQFull + 3, kSFree1 = kQFull + 4;
   static constexpr int kPFull = kQFull + 5, kPvDone = kQFull + 6, kOFull = kQFull + 7;
   static constexpr int kLanded0 = kQFull + 8;                      // FP8: codes in the stage
-  static constexpr int kNumBars = kLanded0 + (kFp8 ? kStages : 0);
+  static constexpr int kDrain0 = kLanded0 + (kFp8 ? kStages : 0);  // MMA drain after an abort
+  static constexpr int kNumBars = kDrain0 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem address + abort flag
   static constexpr int kSmemUsed = kOffMisc + 16;
   static constexpr int kSmemBytes = kSmemUsed + 1024;      // slack to align the base to 1024 B
@@ -135,8 +136,9 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
 
 // Bounded wait whose outcome is the same for every lane of the warp, so that
 // warp-collective TMEM accesses that follow are reached by all lanes or none.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort, kWaitLimitNs);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -184,6 +186,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   grid_dependency_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int worker = blockIdx.x, rb = blockIdx.y;
+  const uint64_t wait_ns = p.wait_ns;  // limit of every bounded wait (normally kWaitLimitNs)
   const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
   const int npieces = md[5];
   if (npieces == 0) return;  // idle worker: uniform exit before any barrier or TMEM use
@@ -208,6 +211,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if constexpr (kFp8) {
       for (int s = 0; s < kStages; ++s) mbar_init(&bar[C::kLanded0 + s], 1);
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[C::kDrain0 + i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -251,7 +255,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int e = -1; e < pz.npg; ++e) {
           const int stage = entries % kStages, use = entries / kStages;
           if (use > 0) {
-            ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, kWaitLimitNs);
+            ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
           }
           uint8_t* dst = skv + stage * kTileBytes;
@@ -286,11 +290,9 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // entry reused its stage.
       for (int s = 0; s < kStages; ++s)
         if ((landed_used >> s) & 1)
-          mbar_wait(&bar[C::kLanded0 + s], ((landed_parity >> s) & 1) ^ 1, abort_flag,
-                    kWaitLimitNs);
+          mbar_wait_drain(&bar[C::kLanded0 + s], ((landed_parity >> s) & 1) ^ 1, kWaitLimitNs);
       if (last_q >= 0 && last_q >= entries - kStages)
-        mbar_wait(&bar[kFull0 + last_q % kStages], (last_q / kStages) & 1, abort_flag,
-                  kWaitLimitNs);
+        mbar_wait_drain(&bar[kFull0 + last_q % kStages], (last_q / kStages) & 1, kWaitLimitNs);
     }
   } else if (kFp8 && warp >= kConvWarp0) {
     // ------------------------------------------------------------ FP8 converters
@@ -319,7 +321,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int stage = entries % kStages;
         const uint32_t parity = (landed_parity >> stage) & 1;
         landed_parity ^= 1u << stage;
-        warp_wait(&bar[C::kLanded0 + stage], parity, abort_flag);  // gives up at once on abort
+        warp_wait(&bar[C::kLanded0 + stage], parity, abort_flag, wait_ns);  // gives up at once on abort
         named_bar_sync(kConvBarrier, kConvThreads);
         if (*abort_flag) { stop = true; break; }
         uint8_t* tile = skv + stage * kTileBytes;
@@ -374,7 +376,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int e = -1; e < pz.npg; ++e) {  // e = -1: the query rows
           const int stage = entries % kStages, use = entries / kStages;
           if (use > 0) {
-            ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, kWaitLimitNs);
+            ok = mbar_wait(&bar[kEmpty0 + stage], (use - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
           }
           uint8_t* dst = skv + stage * kTileBytes;
@@ -393,7 +395,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // Before leaving, let every copy this thread issued land (bounded).
       for (int s = 0; s < kStages && s < entries; ++s) {
         const int n = entries - 1 - s;
-        mbar_wait(&bar[kFull0 + n % kStages], (n / kStages) & 1, abort_flag, kWaitLimitNs);
+        mbar_wait_drain(&bar[kFull0 + n % kStages], (n / kStages) & 1, kWaitLimitNs);
       }
     }
   } else if (warp == kMmaWarp || warp == kQkOddWarp) {
@@ -413,7 +415,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int q_entry = entries;   // copied into TMEM by the softmax warps
         const int first = entries + 1;
         entries += 1 + pz.npg;
-        ok = mbar_wait(&bar[kQFull], qloads & 1, abort_flag, kWaitLimitNs);
+        ok = mbar_wait(&bar[kQFull], qloads & 1, abort_flag, wait_ns);
         ++qloads;
         if (!ok) break;
         if (parity == 0) mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // query stage free
@@ -422,11 +424,11 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int g = pages + j, b = g & 1;
           if (b != parity) continue;
           if (g >= 2) {  // the softmax has read S of page g - 2 from buffer b
-            ok = mbar_wait(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag, kWaitLimitNs);
+            ok = mbar_wait(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
           }
           const int entry = first + j, stage = entry % kStages;
-          ok = mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, kWaitLimitNs);
+          ok = mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint64_t b0 = smem_desc_sw128(kv_base + stage * kTileBytes, 16, 1024);
@@ -457,7 +459,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int g = pages + j;
           // P of page g is in shared memory (and QK^T of page g, which read the
           // same stage, has completed: the softmax saw its S)
-          ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, kWaitLimitNs);
+          ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, wait_ns);
           if (!ok) break;
           tc_fence_after();
           const int stage = (first + j) % kStages;
@@ -519,7 +521,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int q_entry = entries;
         entries += 1 + pz.npg;
         const int qstage = q_entry % kStages;
-        ok = warp_wait(&bar[kFull0 + qstage], (q_entry / kStages) & 1, abort_flag);
+        ok = warp_wait(&bar[kFull0 + qstage], (q_entry / kStages) & 1, abort_flag, wait_ns);
         if (!ok) break;
         {
           const uint8_t* qt = skv + qstage * kTileBytes;
@@ -550,7 +552,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
         for (int j = 0; j < pz.npg; ++j) {
           const int g = pages + j;
-          ok = warp_wait(&bar[kSFull0 + (g & 1)], (g >> 1) & 1, abort_flag);
+          ok = warp_wait(&bar[kSFull0 + (g & 1)], (g >> 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
           tc_fence_after();
           uint32_t s[32];
@@ -603,7 +605,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           l_b = l_b * alpha_b + sum_b;
           // P and O may be touched only after PV of the previous page is done.
           if (j > 0) {
-            ok = warp_wait(&bar[kPvDone], (g - 1) & 1, abort_flag);
+            ok = warp_wait(&bar[kPvDone], (g - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
             tc_fence_after();
             if (__any_sync(0xffffffffu, alpha_a != 1.f || alpha_b != 1.f)) {
@@ -631,7 +633,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           mbar_arrive(&bar[kPFull]);
         }
         if (!ok) break;
-        ok = warp_wait(&bar[kOFull], pieces_done & 1, abort_flag);
+        ok = warp_wait(&bar[kOFull], pieces_done & 1, abort_flag, wait_ns);
         ++pieces_done;
         pages += pz.npg;
         if (!ok) break;
@@ -689,6 +691,17 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   }
 
+  // After an abort, MMAs this CTA issued may still be in flight: each issuing
+  // thread waits for its own through a commit before tensor and shared memory
+  // are released (the TMA producer has already let its copies land).
+  if (*abort_flag) {
+    if (lane == 0 && (warp == kMmaWarp || warp == kPvWarp || warp == kQkOddWarp)) {
+      uint64_t* db = &bar[C::kDrain0 + (warp - kMmaWarp)];
+      umma_commit(db);
+      mbar_wait_drain(db, 0, kWaitLimitNs);
+    }
+    if (threadIdx.x == 0) abort_grace();
+  }
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) report(p.status, MLA_ERR_DEVICE_TIMEOUT);

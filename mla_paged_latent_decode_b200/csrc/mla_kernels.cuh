@@ -36,6 +36,8 @@ struct DecodeParams {
   int batch, s_q, h_q, rows;  // rows = s_q * h_q
   int causal;
   float scale_log2;     // softmax_scale * log2(e)
+  uint64_t wait_ns;     // limit of each bounded device wait (kWaitLimitNs unless lowered
+                        // through mla_set_wait_limit_ns)
 };
 
 struct CombineParams {
@@ -109,9 +111,13 @@ cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_pag
                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
-                               const CUtensorMap& tm_vpart, const CUtensorMap& tm_po,
+                               const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
                                const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
                                cudaStream_t stream);
 cudaError_t pair_kernel_max_clusters(int* clusters);
+// Merge of decode results over disjoint parts of the cache (mla_merge.cu):
+// outs [parts, nrows, 512] bf16, lses [parts, b, h_q, s_q] fp32.
+cudaError_t launch_merge(const void* outs, const float* lses, int parts, int64_t nrows, int s_q,
+                         int h_q, void* out, float* lse, cudaStream_t stream);
 
 }  // namespace mla

@@ -71,6 +71,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that does not give up on an abort: after an abort, a role uses
+// it to let asynchronous work it has already issued (TMA copies, MMAs) finish
+// before the CTA releases the memory that work writes.  Returns false if the
+// limit passed first.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// After an abort: time for TMA copies already in flight to land.  A copy cannot
+// be cancelled, and one lands within microseconds of its issue; where the
+// issuing thread cannot observe its completion (copies counted on the pair
+// leader's barrier), the CTA waits this long before it exits.
+constexpr uint64_t kAbortGraceNs = 200000ull;
+__device__ __forceinline__ void abort_grace() {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < kAbortGraceNs) {
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, uint64_t* bar) {
@@ -481,6 +506,17 @@ __device__ __forceinline__ void umma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tm
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at `bar`'s offset in the pair leader (CTA 0) only,
+// when every pair MMA issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit_leader(uint64_t* bar) {
+  const uint16_t mask = 0x1;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_addr(bar)),
+      "h"(mask)
       : "memory");
 }
 

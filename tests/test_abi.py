@@ -317,3 +317,27 @@ def test_static_scratch_checks_arguments_before_the_limit():
     assert call(batch=0) == binding.MLA_ERR_INVALID_ARG
     # well-formed arguments: the limit is reported, before any device call
     assert call() == binding.MLA_ERR_SCRATCH_LIMIT
+
+
+def test_wait_limit_setting_is_clamped():
+    # the device wait limit (a host-side setting read at each decode launch)
+    assert binding.set_wait_limit_ns(5) == 2_000_000_000
+    assert binding.set_wait_limit_ns(10**12) == 1000       # 5 ns was raised to 1 us
+    assert binding.set_wait_limit_ns(0) == 2_000_000_000   # 10^12 was lowered to 2 s
+    assert binding.set_wait_limit_ns(0) == 2_000_000_000
+
+
+def test_merge_host_validation():
+    lib = binding.lib
+    v = ctypes.c_void_p
+    ok = dict(outs=1 << 12, lses=1 << 12, R=2, b=2, s_q=1, h_q=16, out=1 << 13, lse=1 << 13)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.mla_merge_partials(v(a["outs"]), v(a["lses"]), a["R"], a["b"], a["s_q"],
+                                      a["h_q"], v(a["out"]), v(a["lse"]), v(0))
+    for kw in (dict(outs=0), dict(lses=0), dict(out=0), dict(lse=0), dict(R=0), dict(R=4097),
+               dict(b=0), dict(s_q=0), dict(h_q=0), dict(outs=(1 << 12) + 8),
+               dict(out=(1 << 13) + 8), dict(lse=(1 << 13) + 2), dict(s_q=512, h_q=256),
+               dict(R=4096, b=1 << 16, h_q=128)):
+        assert call(**kw) == binding.MLA_ERR_INVALID_ARG, kw
