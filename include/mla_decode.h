@@ -276,10 +276,12 @@ int mla_append_latent_fp8(const void* rows, int s_new, void* kcache, float* ksca
  * kernel zeroes them), so their codes and scales may hold anything.  Widening
  * is exact for scales 2^k with -124 <= k <= 67 (what the quantising append
  * writes for rows whose largest magnitude lies in about [1e-35, 6.6e22]).
- * Requires s_q * h_q <= 64 query rows per sequence (MLA_ERR_UNSUPPORTED
- * otherwise); metadata from mla_get_metadata as for mla_decode_kvcache.  All
- * other arguments, the workspace, errors and launches are as for
- * mla_decode_kvcache.
+ * Any s_q * h_q up to 65536 (MLA_ERR_UNSUPPORTED above): one CTA per worker
+ * and 64-row block of query rows (the blocks of one worker run side by side and
+ * read the same pages, the second time mostly from L2); metadata from
+ * mla_get_metadata as for mla_decode_kvcache (with more than 64 rows its
+ * worker count keeps every CTA of the grid resident at once).  All other
+ * arguments, the workspace, errors and launches are as for mla_decode_kvcache.
  */
 int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscale,
                            int64_t num_blocks, const int32_t* block_table, int bt_stride,
@@ -393,6 +395,20 @@ int mla_merge_partials(const void* outs, const float* lses, int num_parts, int b
  * thread (a process-wide setting).  Returns the previous limit.
  */
 uint64_t mla_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * mla_debug_set_stall_flag -- test hook of the timeout path.
+ *
+ * Not part of the method.  With a non-null device pointer to an int32 word, the
+ * PV-issuing thread of every decode CTA launched afterwards waits, before its
+ * first PV, for that word to become non-zero (a bounded wait like every other:
+ * mla_set_wait_limit_ns).  A word that stays zero makes that wait run out while
+ * the CTA's TMA copies and QK^T MMAs are in flight, which exercises the drain
+ * and the MLA_ERR_DEVICE_TIMEOUT report.  NULL (the default) switches the hook
+ * off.  Process-wide; the caller owns the word and keeps it alive while such
+ * launches run.  Returns the previous pointer.
+ */
+const int32_t* mla_debug_set_stall_flag(const int32_t* device_flag);
 
 /* mla_version -- build identification string (never NULL). */
 const char* mla_version(void);

@@ -33,6 +33,7 @@ EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_size", "mla_
            "mla_decode_kvcache_static_scratch", "mla_append_latent", "mla_release_pages",
            "mla_append_latent_fp8", "mla_decode_kvcache_fp8", "mla_sparse_workspace_size",
            "mla_decode_sparse", "mla_merge_partials", "mla_set_wait_limit_ns",
+           "mla_debug_set_stall_flag",
            "mla_error_string", "mla_version")
 
 
@@ -81,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.mla_error_string.restype = ctypes.c_char_p
     lib.mla_merge_partials.argtypes = [p, p, i32, i32, i32, i32, p, p, p]
     lib.mla_merge_partials.restype = i32
+    lib.mla_debug_set_stall_flag.argtypes = [p]
+    lib.mla_debug_set_stall_flag.restype = p
     lib.mla_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.mla_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.mla_version.argtypes = []
@@ -98,6 +101,15 @@ def error_string(code: int) -> str:
 
 def version() -> str:
     return lib.mla_version().decode()
+
+
+def debug_set_stall_flag(flag: torch.Tensor | None):
+    """Test hook of the timeout path: the PV issuer of every decode CTA waits for
+    flag (a device int32) to become non-zero before its first PV.  None = off."""
+    if flag is not None:
+        _require(flag.is_cuda and flag.dtype == torch.int32 and flag.numel() >= 1,
+                 "flag must be a device int32")
+    lib.mla_debug_set_stall_flag(_ptr(flag))
 
 
 def set_wait_limit_ns(ns: int) -> int:

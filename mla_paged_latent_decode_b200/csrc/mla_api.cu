@@ -18,6 +18,8 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
 // Limit of each bounded wait inside the decode kernels (mla_set_wait_limit_ns).
 std::atomic<uint64_t> g_wait_ns{mla::kWaitLimitNs};
+// Test hook of the timeout path (mla_debug_set_stall_flag); normally null.
+std::atomic<const int32_t*> g_stall_flag{nullptr};
 
 int current_sm_count(int* sms) {
   int dev = 0;
@@ -204,6 +206,10 @@ uint64_t mla_set_wait_limit_ns(uint64_t ns) {
   return g_wait_ns.exchange(ns);
 }
 
+const int32_t* mla_debug_set_stall_flag(const int32_t* device_flag) {
+  return g_stall_flag.exchange(device_flag);
+}
+
 const char* mla_version(void) {
   return "mla_paged_latent_decode_b200 sm_100a (tcgen05 pair decode for >64 query rows, M=64 decode otherwise)";
 }
@@ -295,6 +301,7 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   p.causal = causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  p.stall_flag = g_stall_flag.load(std::memory_order_relaxed);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (uses_pairs(s_q, h_q)) {
@@ -334,7 +341,7 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   if (batch < 1 || s_q < 1 || h_q < 1 || bt_stride < 1 || num_workers < 1 ||
       num_workers > (1 << 20) || (causal != 0 && causal != 1))
     return MLA_ERR_INVALID_ARG;
-  if (uses_pairs(s_q, h_q)) return MLA_ERR_UNSUPPORTED;  // more than 64 query rows
+  if (static_cast<int64_t>(s_q) * h_q > 65536) return MLA_ERR_UNSUPPORTED;
   if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(batch) * s_q * h_q >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
@@ -373,6 +380,7 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   p.causal = causal;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  p.stall_flag = g_stall_flag.load(std::memory_order_relaxed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mla::launch_decode_fp8(tm_q, tm_page8, p, num_workers, st) != cudaSuccess)
     return MLA_ERR_CUDA;

@@ -458,6 +458,11 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int g = pages + j, slot = entries % kKSlots, pb = g & 1;
           ok = mbar_wait_cluster(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
+          // test hook: a wait that nothing ends, with copies and MMAs in flight
+          if (g == 0 && p.stall_flag != nullptr) {
+            ok = flag_wait(p.stall_flag, abort_flag, wait_ns);
+            if (!ok) break;
+          }
           ok = mbar_wait_cluster(&bar[kVFull0 + slot], (vbits >> slot) & 1u, abort_flag,
                                  wait_ns);
           if (!ok) break;

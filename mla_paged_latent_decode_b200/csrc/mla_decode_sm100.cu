@@ -142,25 +142,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-// E4M3 -> bf16 without the conversion unit (whose throughput is a small
-// fraction of the integer and FMA pipes').  For a code b = s eeee mmm, the
-// 16-bit pattern s 0000 eeee mmm 0000 is the bf16 value b * 2^-120 (E4M3
-// subnormals become bf16 subnormals, zero stays zero).  Two exact bf16x2
-// multiplies, by 2^60 and by 2^60 * scale, then give b * scale: every step is
-// exact for scales 2^k with -124 <= k <= 67 (below -124 the smallest codes
-// times the scale fall under bf16's range).
-//   bytes2: the two codes sit in bytes sel selects (0x1404: bytes 0, 1;
-//   0x3424: bytes 2, 3); lo code -> low half.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t word, uint32_t sel,
-                                                     uint32_t f_hi, uint32_t f_lo) {
-  const uint32_t t = __byte_perm(word, 0u, sel);  // (b_hi << 24) | (b_lo << 8)
-  const uint32_t pat = ((t & 0x7F007F00u) >> 4) | (t & 0x80008000u);
-  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pat);
-  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_hi));
-  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_lo));
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
 template <bool kFp8>
 __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -461,6 +442,11 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // same stage, has completed: the softmax saw its S)
           ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, wait_ns);
           if (!ok) break;
+          // test hook: a wait that nothing ends, with copies and MMAs in flight
+          if (g == 0 && p.stall_flag != nullptr) {
+            ok = flag_wait(p.stall_flag, abort_flag, wait_ns);
+            if (!ok) break;
+          }
           tc_fence_after();
           const int stage = (first + j) % kStages;
           const uint32_t tile = kv_base + stage * kTileBytes;

@@ -38,6 +38,8 @@ struct DecodeParams {
   float scale_log2;     // softmax_scale * log2(e)
   uint64_t wait_ns;     // limit of each bounded device wait (kWaitLimitNs unless lowered
                         // through mla_set_wait_limit_ns)
+  const int32_t* stall_flag;  // test hook, normally null: when set, the PV issuer waits
+                              // for it to become non-zero before its first PV
 };
 
 struct CombineParams {

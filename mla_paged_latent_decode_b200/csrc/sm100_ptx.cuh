@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cstdint>
 
 namespace mla {
@@ -82,6 +83,23 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Bounded wait for a word in global memory to become non-zero (the same
+// give-up rules as mbar_wait).
+__device__ __forceinline__ bool flag_wait(const volatile int32_t* flag, volatile int* abort,
+                                          uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (*flag != 0) return true;
+    if ((it & 15u) == 15u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        return false;
+      }
+    }
   }
 }
 
@@ -399,6 +417,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// E4M3 -> bf16 without the conversion unit (whose throughput is a small
+// fraction of the integer and FMA pipes').  For a code b = s eeee mmm, the
+// 16-bit pattern s 0000 eeee mmm 0000 is the bf16 value b * 2^-120 (E4M3
+// subnormals become bf16 subnormals, zero stays zero).  Two exact bf16x2
+// multiplies, by 2^60 and by 2^60 * scale, then give b * scale: every step is
+// exact for scales 2^k with -124 <= k <= 67 (below -124 the smallest codes
+// times the scale fall under bf16's range).
+//   bytes2: the two codes sit in bytes sel selects (0x1404: bytes 0, 1;
+//   0x3424: bytes 2, 3); lo code -> low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t word, uint32_t sel,
+                                                     uint32_t f_hi, uint32_t f_lo) {
+  const uint32_t t = __byte_perm(word, 0u, sel);  // (b_hi << 24) | (b_lo << 8)
+  const uint32_t pat = ((t & 0x7F007F00u) >> 4) | (t & 0x80008000u);
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pat);
+  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_hi));
+  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f_lo));
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // ---------------------------------------------------------------- CTA pairs (clusters of 2)

@@ -160,8 +160,7 @@ def _fp8_decode_raw(**kw):
     (dict(kscale=0), binding.MLA_ERR_INVALID_ARG),
     (dict(kcache=0), binding.MLA_ERR_INVALID_ARG),
     (dict(kscale=(1 << 12) + 4), binding.MLA_ERR_INVALID_ARG),
-    (dict(h_q=128), binding.MLA_ERR_UNSUPPORTED),      # more than 64 query rows
-    (dict(s_q=2, h_q=64), binding.MLA_ERR_UNSUPPORTED),
+    (dict(s_q=2, h_q=65536), binding.MLA_ERR_UNSUPPORTED),   # more than 65536 query rows
     (dict(d=512), binding.MLA_ERR_UNSUPPORTED),
     (dict(causal=3), binding.MLA_ERR_INVALID_ARG),
     (dict(workspace_bytes=64), binding.MLA_ERR_INVALID_ARG),

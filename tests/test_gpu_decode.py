@@ -29,6 +29,24 @@ def test_small_shapes(cuda_device, h_q, s_q, causal):
     full_parity(inp, cuda_device)
 
 
+@pytest.mark.parametrize("s_q,h_q,causal", [(1, 1, False), (1, 4, False), (2, 8, True),
+                                             (1, 16, False), (4, 4, True), (3, 5, False)])
+def test_narrow_rows(cuda_device, s_q, h_q, causal):
+    # few query rows per sequence (1 to 16): most of the single-CTA kernel's
+    # 64-row block is padding, whose rows must never reach the output
+    w = synth.custom_workload(5, s_q, h_q, [1, 63, 64, 130, 2000], causal=causal)
+    inp = synth.make_inputs(w, seed=400 + s_q * h_q)
+    full_parity(inp, cuda_device)
+    full_parity(inp, cuda_device, num_workers=9)
+
+
+@pytest.mark.parametrize("num_workers", [1, 2, 7, 148, 600])
+def test_few_rows_forced_splits_and_poison(cuda_device, num_workers):
+    w = synth.custom_workload(3, 1, 16, [700, 5, 1100])
+    inp = synth.make_inputs(w, seed=17, poison=True)
+    full_parity(inp, cuda_device, num_workers=num_workers)
+
+
 @pytest.mark.parametrize("num_workers", [1, 3, 17, 148, 600])
 def test_forced_splits(cuda_device, num_workers):
     # num_workers controls how finely sequences are cut: 1 = no splits at all,

@@ -74,6 +74,36 @@ def test_fp8_decode_small(cuda_device, h_q, s_q, causal):
     assert_close_lse(lse, ref_lse, "fp8 lse")
 
 
+@pytest.mark.parametrize("h_q,s_q,causal", [(128, 1, False), (128, 2, True), (96, 1, False),
+                                             (64, 3, True)])
+def test_fp8_decode_more_than_64_rows(cuda_device, h_q, s_q, causal):
+    # several 64-row blocks per worker, a last block with some or no valid rows
+    w = synth.custom_workload(4, s_q, h_q, [1, 63, 700, 1300], causal=causal)
+    inp = synth.make_inputs(w, seed=310 + h_q + s_q)
+    codes, scales = encode_cache(inp.kcache)
+    for nw in (None, 5):
+        out, lse, md, ns = run_fp8(inp, codes, scales, cuda_device, nw)
+        check_metadata(inp, dict(tile_md=md, num_splits=ns), md.shape[0])
+        ref_out, ref_lse = oracle.decode(inp.q, dequantized(codes, scales), inp.block_table,
+                                         inp.cache_seqlens, inp.scale, inp.causal)
+        assert_close_out(out, ref_out, "fp8 out")
+        assert_close_lse(lse, ref_lse, "fp8 lse")
+
+
+@pytest.mark.parametrize("name", ["dsv3_decode", "spec_causal", "skewed_long"])
+def test_fp8_full_size_128_heads(cuda_device, name):
+    # the 128-head configurations over their FP8 caches, default launch
+    # configuration, every element against the oracle on the dequantised cache
+    inp = synth.make_inputs(name, seed=0)
+    codes, scales = encode_cache(inp.kcache)
+    out, lse, md, ns = run_fp8(inp, codes, scales, cuda_device)
+    check_metadata(inp, dict(tile_md=md, num_splits=ns), md.shape[0])
+    ref_out, ref_lse = oracle.decode(inp.q, dequantized(codes, scales), inp.block_table,
+                                     inp.cache_seqlens, inp.scale, inp.causal)
+    assert_close_out(out, ref_out, "fp8 out")
+    assert_close_lse(lse, ref_lse, "fp8 lse")
+
+
 @pytest.mark.parametrize("num_workers", [1, 3, 17, 600])
 def test_fp8_decode_forced_splits(cuda_device, num_workers):
     w = synth.custom_workload(3, 2, 16, [700, 5, 1100], causal=True)
