@@ -312,10 +312,10 @@ int mla_release_pages(const int32_t* release_mask, int32_t* block_table, int bt_
 
 /*
  * mla_sparse_workspace_size -- bytes of workspace mla_decode_sparse needs:
- * the compacted index lists, the gathered rows (ceil(topk / 64) pages of 64
- * rows x 1152 bytes per query position), the split metadata and partials of
- * the decode over them.  num_workers: mla_metadata_shape(batch * s_q, h_q, 1).
- * Returns 0 for invalid arguments.
+ * the cached row of every used index entry (4 bytes per entry and query
+ * position), the counts, and the split metadata and partials of the decode
+ * over them.  num_workers: mla_metadata_shape(batch * s_q, h_q, 1).  Returns 0
+ * for invalid arguments.
  */
 size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int num_workers);
 
@@ -340,10 +340,12 @@ size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int num_
  * Requires topk <= 65536, batch * s_q <= 65536.  A used entry whose page lies
  * outside the block-table row or the cache is read as a zero row and reported
  * as MLA_ERR_DEVICE_CHECK in device_status.
- * Launches: a compaction kernel and a gather kernel (each used entry's row is
- * copied into workspace pages, one sequence per query position), then the
- * scheduler, decode and combine kernels of mla_decode_kvcache over them, and
- * (s_q > 1) a kernel that reorders lse.  No host synchronisation.
+ * Launches: a compaction kernel (the used entries of each query position, as
+ * cached rows, in list order), then the scheduler, decode and combine kernels
+ * of mla_decode_kvcache over b * s_q sequences of one query position each,
+ * the decode kernel copying the listed rows from the cache itself (each
+ * selected row is read once), and (s_q > 1) a kernel that reorders lse.  No
+ * host synchronisation.
  */
 int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
                       const int32_t* block_table, int bt_stride, const int32_t* cache_seqlens,

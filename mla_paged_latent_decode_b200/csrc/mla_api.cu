@@ -161,6 +161,76 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int launch_combine_for(const int32_t* num_splits, float* part_o, float* part_lse, void* out,
                        float* lse, int batch, int s_q, int h_q, int rows, cudaStream_t st);
 
+// The decode after argument checks: scheduler metadata given, workspace large
+// enough.  gather_rows != null: the rows of sequence s are cached rows
+// gather_rows[s * gather_stride + k] (CTA pairs only; block_table unused).
+int decode_impl(const void* q, const void* kcache, int64_t num_blocks, const int32_t* block_table,
+                int bt_stride, const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dv,
+                float softmax_scale, int causal, const int32_t* tile_md, const int32_t* num_splits,
+                int num_workers, void* workspace, void* out, float* lse, int32_t* device_status,
+                void* stream, const int32_t* gather_rows, int64_t gather_stride) {
+  const int rows = s_q * h_q;
+  CUtensorMap tm_q;
+  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
+  const uint64_t cache_rows = static_cast<uint64_t>(num_blocks) * mla::kPage;
+
+  const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             round_up(slots * rows * dv * sizeof(float), 256));
+
+  mla::DecodeParams p{};
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.status = device_status;
+  p.bt_stride = bt_stride;
+  p.num_blocks = num_blocks;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = rows;
+  p.causal = causal;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  p.stall_flag = g_stall_flag.load(std::memory_order_relaxed);
+  p.gather_rows = gather_rows;
+  p.gather_cache = kcache;
+  p.gather_stride = gather_stride;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (uses_pairs(s_q, h_q)) {
+    // K part: 32 token rows x all 9 chunks per box; peer-token values: 32 rows x 4
+    // chunks (gathered rows are copied without these maps)
+    CUtensorMap tm_kpart = tm_q, tm_vx = tm_q;
+    if (gather_rows == nullptr) {
+      if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, mla::kDqk / 64)) return MLA_ERR_CUDA;
+      if (!make_chunk_map(&tm_vx, kcache, cache_rows, 32, 4)) return MLA_ERR_CUDA;
+    }
+    CUtensorMap tm_po, tm_out;
+    if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
+    if (!make_out_map(&tm_out, out, static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)))
+      return MLA_ERR_CUDA;
+    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vx, tm_po, tm_out, p, num_workers, st) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
+  } else {
+    // a whole page (64 rows x 9 chunks) per box (gathered rows are copied without it)
+    CUtensorMap tm_page = tm_q;
+    if (gather_rows == nullptr &&
+        !make_chunk_map(&tm_page, kcache, cache_rows, 64, mla::kDqk / 64))
+      return MLA_ERR_CUDA;
+    if (mla::launch_decode(tm_q, tm_page, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+
+  return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -272,58 +342,9 @@ int mla_decode_kvcache(const void* q, const void* kcache, int64_t num_blocks,
   const size_t need = mla_workspace_size(batch, s_q, h_q, dv, num_workers);
   if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
 
-  const int rows = s_q * h_q;
-  CUtensorMap tm_q;
-  if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
-  const uint64_t cache_rows = static_cast<uint64_t>(num_blocks) * mla::kPage;
-
-  const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
-  float* part_o = static_cast<float*>(workspace);
-  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                             round_up(slots * rows * dv * sizeof(float), 256));
-
-  mla::DecodeParams p{};
-  p.block_table = block_table;
-  p.seqlens = cache_seqlens;
-  p.tile_md = tile_md;
-  p.num_splits = num_splits;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.part_o = part_o;
-  p.part_lse = part_lse;
-  p.status = device_status;
-  p.bt_stride = bt_stride;
-  p.num_blocks = num_blocks;
-  p.batch = batch;
-  p.s_q = s_q;
-  p.h_q = h_q;
-  p.rows = rows;
-  p.causal = causal;
-  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
-  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
-  p.stall_flag = g_stall_flag.load(std::memory_order_relaxed);
-
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (uses_pairs(s_q, h_q)) {
-    // K part: 32 token rows x all 9 chunks per box; peer-token values: 32 rows x 4 chunks
-    CUtensorMap tm_kpart, tm_vx;
-    if (!make_chunk_map(&tm_kpart, kcache, cache_rows, 32, mla::kDqk / 64)) return MLA_ERR_CUDA;
-    if (!make_chunk_map(&tm_vx, kcache, cache_rows, 32, 4)) return MLA_ERR_CUDA;
-    CUtensorMap tm_po, tm_out;
-    if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
-    if (!make_out_map(&tm_out, out, static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)))
-      return MLA_ERR_CUDA;
-    if (mla::launch_decode_pair(tm_q, tm_kpart, tm_vx, tm_po, tm_out, p, num_workers, st) !=
-        cudaSuccess)
-      return MLA_ERR_CUDA;
-  } else {
-    // a whole page (64 rows x 9 chunks) per box
-    CUtensorMap tm_page;
-    if (!make_chunk_map(&tm_page, kcache, cache_rows, 64, mla::kDqk / 64)) return MLA_ERR_CUDA;
-    if (mla::launch_decode(tm_q, tm_page, p, num_workers, st) != cudaSuccess) return MLA_ERR_CUDA;
-  }
-
-  return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
+  return decode_impl(q, kcache, num_blocks, block_table, bt_stride, cache_seqlens, batch, s_q,
+                     h_q, dv, softmax_scale, causal, tile_md, num_splits, num_workers, workspace,
+                     out, lse, device_status, stream, nullptr, 0);
 }
 
 int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscale,
@@ -390,13 +411,11 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
 size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int topk, int num_workers) {
   if (batch < 1 || s_q < 1 || h_q < 1 || topk < 1 || num_workers < 1) return 0;
   const size_t pos = static_cast<size_t>(batch) * s_q;
-  const size_t ppp = (static_cast<size_t>(topk) + mla::kPage - 1) / mla::kPage;
   const size_t dec = mla_workspace_size(static_cast<int>(pos), 1, h_q, mla::kDv, num_workers);
   if (dec == 0) return 0;
-  return round_up(pos * topk * 4, 256) + round_up(pos * 4, 256) + round_up(pos * ppp * 4, 256) +
+  return round_up(pos * topk * 4, 256) + round_up(pos * 4, 256) +
          round_up(static_cast<size_t>(num_workers) * MLA_MD_STRIDE * 4, 256) +
-         round_up((pos + 1) * 4, 256) + round_up(pos * h_q * 4, 256) + dec +
-         pos * ppp * mla::kPage * mla::kDqk * 2;
+         round_up((pos + 1) * 4, 256) + round_up(pos * h_q * 4, 256) + dec;
 }
 
 int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
@@ -416,8 +435,7 @@ int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
   if (num_blocks < 1 || num_blocks * mla::kPage >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
   const int64_t pos = static_cast<int64_t>(batch) * s_q;
   const int64_t ppp = (topk + mla::kPage - 1) / mla::kPage;
-  if (pos > 65536 || pos * ppp * mla::kPage >= (int64_t(1) << 31) ||
-      pos * h_q >= (int64_t(1) << 31))
+  if (pos > 65536 || pos * topk >= (int64_t(1) << 31) || pos * h_q >= (int64_t(1) << 31))
     return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
@@ -436,16 +454,12 @@ int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
   sp.indices = indices;
   sp.seqlens = cache_seqlens;
   sp.block_table = block_table;
-  sp.kcache = kcache;
   sp.comp = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos) * topk * 4));
   sp.counts = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos) * 4));
-  sp.comp_bt = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos * ppp) * 4));
   int32_t* tile_md = reinterpret_cast<int32_t*>(take(static_cast<size_t>(num_workers) * MLA_MD_STRIDE * 4));
   int32_t* num_splits = reinterpret_cast<int32_t*>(take(static_cast<size_t>(pos + 1) * 4));
   float* lse_pos = reinterpret_cast<float*>(take(static_cast<size_t>(pos) * h_q * 4));
-  const size_t dec_bytes = mla_workspace_size(static_cast<int>(pos), 1, h_q, mla::kDv, num_workers);
-  void* dec_ws = take(dec_bytes);
-  sp.comp_cache = w;  // the rest: the gathered pages
+  void* dec_ws = take(mla_workspace_size(static_cast<int>(pos), 1, h_q, mla::kDv, num_workers));
   sp.status = device_status;
   sp.bt_stride = bt_stride;
   sp.num_blocks = num_blocks;
@@ -453,17 +467,18 @@ int mla_decode_sparse(const void* q, const void* kcache, int64_t num_blocks,
   sp.s_q = s_q;
   sp.topk = topk;
   sp.causal = causal;
-  sp.pages_per_pos = static_cast<int>(ppp);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mla::launch_sparse_prepare(sp, st) != cudaSuccess) return MLA_ERR_CUDA;
   int rc = mla_get_metadata(sp.counts, static_cast<int>(pos), h_q, 1, tile_md, num_splits,
                             num_workers, stream);
   if (rc != MLA_OK) return rc;
-  rc = mla_decode_kvcache(q, sp.comp_cache, pos * ppp, sp.comp_bt, static_cast<int>(ppp),
-                          sp.counts, static_cast<int>(pos), 1, h_q, d, dv, softmax_scale, 0,
-                          tile_md, num_splits, num_workers, dec_ws, dec_bytes, out,
-                          s_q > 1 ? lse_pos : lse, device_status, stream);
+  // the decode over b * s_q sequences (one query position each) whose rows the
+  // decode kernel copies itself, by index, from the cache
+  float* lse_dst = s_q > 1 ? lse_pos : lse;
+  rc = decode_impl(q, kcache, num_blocks, sp.comp, static_cast<int>(ppp), sp.counts,
+                   static_cast<int>(pos), 1, h_q, dv, softmax_scale, 0, tile_md, num_splits,
+                   num_workers, dec_ws, out, lse_dst, device_status, stream, sp.comp, topk);
   if (rc != MLA_OK) return rc;
   if (s_q > 1 && mla::launch_sparse_lse(lse_pos, lse, batch, s_q, h_q, st) != cudaSuccess)
     return MLA_ERR_CUDA;

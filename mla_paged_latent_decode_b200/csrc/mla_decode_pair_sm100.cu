@@ -218,6 +218,30 @@ __device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar
   return true;
 }
 
+// Gathered rows: copy 32 cached rows (this lane holds the row index of row
+// `lane`; -1 = a zero row) into a slot, chunks src_chunk .. src_chunk +
+// nchunks - 1 of each row to chunks dst_chunk .. of the slot, in the
+// 128-byte-swizzled layout of the TMA boxes.  Lane l copies 16-byte unit l % 8
+// of rows 4 g + l / 8, g = 0..7, so that eight lanes read one 128-byte segment
+// of a row.
+__device__ __forceinline__ void gather_rows32(uint8_t* slot, int dst_chunk, int src_chunk,
+                                              int nchunks, const void* cache, int my_row,
+                                              int lane) {
+  const int u = lane & 7;
+#pragma unroll
+  for (int grp = 0; grp < 8; ++grp) {
+    const int r = 4 * grp + (lane >> 3);
+    const int row = __shfl_sync(0xffffffffu, my_row, r);
+    const uint8_t* src = static_cast<const uint8_t*>(cache) +
+                         static_cast<int64_t>(row < 0 ? 0 : row) * (kDqk * 2) + src_chunk * 128 +
+                         u * 16;
+    uint8_t* dst = slot + dst_chunk * kHalfChunk + r * 128 + ((u ^ (r & 7)) << 4);
+    for (int c = 0; c < nchunks; ++c)
+      cp_async16_zfill(dst + c * kHalfChunk, src + c * 128, row >= 0);
+  }
+}
+
+template <bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kpart,
@@ -227,6 +251,9 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // full barriers of the K and V parts: one TMA-counted arrival (dense pages),
+  // or one arrival per CTA (gathered rows, copied by the threads)
+  constexpr uint32_t kFullArrivals = kGather ? 2 : 1;
   uint8_t* sq2 = smem + kOffQ2;
   uint8_t* sk = smem + kOffK;
   uint8_t* sp = smem + kOffP;
@@ -254,8 +281,8 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKSlots; ++s) {
-      mbar_init(&bar[kKFull0 + s], 1);
-      mbar_init(&bar[kVFull0 + s], 1);
+      mbar_init(&bar[kKFull0 + s], kFullArrivals);
+      mbar_init(&bar[kVFull0 + s], kFullArrivals);
       mbar_init(&bar[kKEmpty0 + s], 1);
       mbar_init(&bar[kXFree0 + 2 * s], 1);
       mbar_init(&bar[kXFree0 + 2 * s + 1], 1);
@@ -293,59 +320,121 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   // two query-staging entries, then one entry per page.
   if (warp == kTmaKWarp) {
     // ------------------------------------------------------------ query rows + K parts
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_kpart);
+    // Dense pages: lane 0 issues one TMA box per page.  Gathered rows (kGather):
+    // all 32 lanes copy the page's 32 rows of this CTA in 16-byte pieces, and a
+    // page is signalled once two newer pages have been issued (up to three
+    // pages of copies in flight), a piece's last pages at the piece's end.
+    if (kGather || lane == 0) {
+      if (lane == 0) {
+        prefetch_tensormap(&tm_q);
+        if (!kGather) prefetch_tensormap(&tm_kpart);
+      }
+      // a wait of the lanes running this loop, with the same outcome in each
+      auto wait = [&](uint64_t* b, uint32_t parity) {
+        bool r = mbar_wait_cluster(b, parity, abort_flag, wait_ns);
+        if constexpr (kGather) r = __all_sync(0xffffffffu, r);
+        return r;
+      };
       int entries = 0, qloads = 0;
+      int pending[2] = {-1, -1};  // gather: slots of the two newest pages not yet signalled
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
-        if (rank == 0 && p.seqlens[pz.seq] > p.bt_stride * kPage)
+        if (lane == 0 && rank == 0 && p.seqlens[pz.seq] > p.bt_stride * kPage)
           report(p.status, MLA_ERR_DEVICE_CHECK);
         if (pz.npg == 0) continue;
         const int qrow = pz.seq * p.rows + row0;
         // dims 384..575 of the query rows: shared memory, counted on the leader
         if (qloads > 0) {
-          ok = mbar_wait_cluster(&bar[kQEmpty], (qloads - 1) & 1, abort_flag, wait_ns);
+          ok = wait(&bar[kQEmpty], (qloads - 1) & 1);
           if (!ok) break;
         }
-        if (rank == 0) mbar_arrive_expect_tx(&bar[kQFull], 2 * kQ2Bytes);
-        for (int c = 0; c < kQSmemChunks; ++c)
-          tma_load_2d_pair(sq2 + c * kChunk, &tm_q, (kQTmemChunks + c) * 64, qrow, &bar[kQFull]);
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive_expect_tx(&bar[kQFull], 2 * kQ2Bytes);
+          for (int c = 0; c < kQSmemChunks; ++c)
+            tma_load_2d_pair(sq2 + c * kChunk, &tm_q, (kQTmemChunks + c) * 64, qrow,
+                             &bar[kQFull]);
+        }
         ++qloads;
         // dims 0..383: two staging entries of the K ring, counted on this CTA's barrier
         for (int e = 0; e < 2; ++e) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
-          if (use > 0)
-            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
-                                   wait_ns);
+          if (use > 0) ok = wait(&bar[kKEmpty0 + slot], (use - 1) & 1);
           if (!ok) break;
-          if (e == 0) mbar_arrive_expect_tx(&bar[kQStage], kQTmemChunks * kChunk);
-          uint8_t* dst = sk + slot * kKBytes;
-          const int c0 = e == 0 ? 0 : kQStageA, c1 = e == 0 ? kQStageA : kQTmemChunks;
-          for (int c = c0; c < c1; ++c)
-            tma_load_2d(dst + (c - c0) * kChunk, &tm_q, c * 64, qrow, &bar[kQStage]);
-          // the leader's full barrier of the slot completes one phase per entry
-          if (rank == 0) mbar_arrive(&bar[kKFull0 + slot]);
+          if (lane == 0) {
+            if (e == 0) mbar_arrive_expect_tx(&bar[kQStage], kQTmemChunks * kChunk);
+            uint8_t* dst = sk + slot * kKBytes;
+            const int c0 = e == 0 ? 0 : kQStageA, c1 = e == 0 ? kQStageA : kQTmemChunks;
+            for (int c = c0; c < c1; ++c)
+              tma_load_2d(dst + (c - c0) * kChunk, &tm_q, c * 64, qrow, &bar[kQStage]);
+            // the leader's full barrier of the slot completes one phase per entry
+            if (rank == 0)
+              for (int a = 0; a < kFullArrivals; ++a) mbar_arrive(&bar[kKFull0 + slot]);
+          }
           ++entries;
         }
         if (!ok) break;
-        const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+        // gather: row of this lane's token (tokens 32 rank .. 32 rank + 31) of a
+        // piece page, loaded one page ahead of its copies
+        const int cnt = kGather ? p.seqlens[pz.seq] : 0;
+        const int32_t* grows =
+            kGather ? p.gather_rows + static_cast<int64_t>(pz.seq) * p.gather_stride : nullptr;
+        auto row_of = [&](int jj) {
+          const int vt0 = (pz.pg0 + jj) * kPage;
+          const int tok = vt0 + 32 * static_cast<int>(rank) + lane;
+          return tok < cnt ? __ldg(grows + tok) : -1;  // past the count: a zero row
+        };
+        int next_row = kGather ? row_of(0) : 0;
         for (int j = 0; j < pz.npg && ok; ++j, ++entries) {
           const int slot = entries % kKSlots, use = entries / kKSlots;
-          const int page = __ldg(bt + pz.pg0 + j);
-          if (use > 0) {
-            ok = mbar_wait_cluster(&bar[kKEmpty0 + slot], (use - 1) & 1, abort_flag,
-                                   wait_ns);
-            if (!ok) break;
+          if constexpr (kGather) {
+            const int my_row = next_row;
+            if (j + 1 < pz.npg) next_row = row_of(j + 1);
+            if (use > 0) {
+              ok = wait(&bar[kKEmpty0 + slot], (use - 1) & 1);
+              if (!ok) break;
+            }
+            gather_rows32(sk + slot * kKBytes, 0, 0, kChunks, p.gather_cache, my_row, lane);
+            cp_async_commit();
+            // two pages of copies stay in flight behind the newest: signal the
+            // page issued two pages ago once its copies have landed
+            if (pending[0] >= 0) {
+              cp_async_wait_group<2>();
+              fence_proxy_async_smem();
+              warp_arrive_leader(&bar[kKFull0 + pending[0]], rank, lane);
+            }
+            pending[0] = pending[1];
+            pending[1] = slot;
+            if (j + 1 == pz.npg) {
+              // the piece's last pages: signal them now (the next piece's query rows
+              // reach the MMAs only after this piece is finished)
+              cp_async_wait_group<0>();
+              fence_proxy_async_smem();
+              for (int k = 0; k < 2; ++k)
+                if (pending[k] >= 0) warp_arrive_leader(&bar[kKFull0 + pending[k]], rank, lane);
+              pending[0] = pending[1] = -1;
+            }
+          } else {
+            const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+            const int page = __ldg(bt + pz.pg0 + j);
+            if (use > 0) {
+              ok = wait(&bar[kKEmpty0 + slot], (use - 1) & 1);
+              if (!ok) break;
+            }
+            // the slot's previous entry is consumed, so the leader's full barrier is
+            // in the phase of this entry
+            if (rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
+            // one box: this CTA's 32 token rows x all nine chunks
+            tma_load_3d_pair(sk + slot * kKBytes, &tm_kpart, 0,
+                             page * kPage + 32 * static_cast<int>(rank), 0,
+                             &bar[kKFull0 + slot]);
           }
-          // the slot's previous entry is consumed, so the leader's full barrier is
-          // in the phase of this entry
-          if (rank == 0) mbar_arrive_expect_tx(&bar[kKFull0 + slot], 2 * kKBytes);
-          // one box: this CTA's 32 token rows x all nine chunks
-          tma_load_3d_pair(sk + slot * kKBytes, &tm_kpart, 0,
-                           page * kPage + 32 * static_cast<int>(rank), 0, &bar[kKFull0 + slot]);
         }
+      }
+      if constexpr (kGather) {
+        // no copy may still be in flight when the CTA releases its shared memory
+        // (after an abort the loop may have left pages unsignalled; nothing reads them)
+        cp_async_wait_group<0>();
       }
     }
   } else if (warp == kTmaVWarp) {
@@ -353,8 +442,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // CTA 0 replaces chunks 4..7 of each page's slot with tokens 32..63 x dims
     // 0..255, CTA 1 chunks 0..3 with tokens 0..31 x dims 256..511, each once the
     // QK^T MMAs have read the chunks being replaced (of both CTAs: one commit).
-    if (lane == 0) {
-      prefetch_tensormap(&tm_vx);
+    // Dense pages: one TMA box (lane 0).  Gathered rows: all lanes copy the
+    // peer tokens' rows and signal the page once their copies have landed.
+    if (kGather || lane == 0) {
+      if (!kGather) prefetch_tensormap(&tm_vx);
       const int xgrp = rank == 0 ? 1 : 0;
       const int dst_chunk = rank == 0 ? kXChunks : 0;
       const int src_row = rank == 0 ? 32 : 0, src_chunk = rank == 0 ? 0 : kXChunks;
@@ -365,21 +456,39 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (pz.npg == 0) continue;
         entries += 2;  // the piece's query staging entries
-        const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
         for (int j = 0; j < pz.npg; ++j, ++entries) {
           const int slot = entries % kKSlots;
-          const int page = __ldg(bt + pz.pg0 + j);
+          int my_row = 0;
+          if constexpr (kGather) {
+            const int vt0 = (pz.pg0 + j) * kPage, cnt = p.seqlens[pz.seq];
+            const int32_t* rows = p.gather_rows + static_cast<int64_t>(pz.seq) * p.gather_stride;
+            const int tok = vt0 + src_row + lane;
+            my_row = tok < cnt ? __ldg(rows + tok) : -1;  // past the count: a zero row
+          }
           ok = mbar_wait_cluster(&bar[kXFree0 + 2 * slot + xgrp], (xbits >> slot) & 1u, abort_flag,
                                  wait_ns);
+          if constexpr (kGather) ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           xbits ^= 1u << slot;
-          // the PV of the slot's previous page is done (its K part was reloaded
-          // after it), so the leader's V barrier is in the phase of this page
-          if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kXBytes);
-          tma_load_3d_pair(sk + slot * kKBytes + dst_chunk * kHalfChunk, &tm_vx, 0,
-                           page * kPage + src_row, src_chunk, &bar[kVFull0 + slot]);
+          if constexpr (kGather) {
+            gather_rows32(sk + slot * kKBytes, dst_chunk, src_chunk, kXChunks, p.gather_cache,
+                          my_row, lane);
+            cp_async_commit();
+            cp_async_wait_group<0>();
+            fence_proxy_async_smem();
+            warp_arrive_leader(&bar[kVFull0 + slot], rank, lane);
+          } else {
+            const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+            const int page = __ldg(bt + pz.pg0 + j);
+            // the PV of the slot's previous page is done (its K part was reloaded
+            // after it), so the leader's V barrier is in the phase of this page
+            if (rank == 0) mbar_arrive_expect_tx(&bar[kVFull0 + slot], 2 * kXBytes);
+            tma_load_3d_pair(sk + slot * kKBytes + dst_chunk * kHalfChunk, &tm_vx, 0,
+                             page * kPage + src_row, src_chunk, &bar[kVFull0 + slot]);
+          }
         }
       }
+      if constexpr (kGather) cp_async_wait_group<0>();
     }
   } else if (warp == kQkEvenWarp || warp == kQkOddWarp) {
     // ------------------------------------------------------------ QK^T issuers (leader)
@@ -777,14 +886,17 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
                                const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
                                const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
                                cudaStream_t stream) {
-  static std::atomic<bool> configured[64];  // per device: attribute set
+  static std::atomic<bool> configured[64];  // per device: attribute set (both variants)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
+    e = cudaFuncSetAttribute(mla_decode_pair_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(mla_decode_pair_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev].store(true, std::memory_order_release);
   }
@@ -803,7 +915,12 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, tm_q, tm_kpart, tm_vx, tm_po, tm_out, p);
+  if (p.gather_rows != nullptr)
+    e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel<true>, tm_q, tm_kpart, tm_vx, tm_po,
+                           tm_out, p);
+  else
+    e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel<false>, tm_q, tm_kpart, tm_vx, tm_po,
+                           tm_out, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -820,8 +937,8 @@ cudaError_t pair_kernel_max_clusters(int* clusters) {
     *clusters = known;
     return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(mla_decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes);
+  e = cudaFuncSetAttribute(mla_decode_pair_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
@@ -835,7 +952,7 @@ cudaError_t pair_kernel_max_clusters(int* clusters) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel<false>, &cfg);
   if (e != cudaSuccess) return e;
   if (n < 1) n = 1;
   cached[dev].store(n, std::memory_order_release);

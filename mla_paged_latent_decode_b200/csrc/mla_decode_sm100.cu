@@ -142,7 +142,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kGather = false>
 __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_page, const DecodeParams p) {
@@ -342,6 +342,92 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (stop) break;
     }
+  } else if (kGather && warp == kTmaWarp) {
+    // ------------------------------------------------------------ gather producer
+    // The sparse decode's rows: token k of sequence s is cached row
+    // gather_rows[s * gather_stride + k].  The query rows come by TMA as in the
+    // dense producer (lane 0); a page's 64 rows are copied by all 32 lanes in
+    // 16-byte pieces (eight lanes per 128-byte row segment) into the same
+    // swizzled tile layout.  Each lane waits for its own copies, issues a proxy
+    // fence, and lane 0 signals the page once the next page has been issued
+    // (one page of copies in flight behind the newest; a piece's last page at
+    // the piece's end).
+    prefetch_tensormap(&tm_q);
+    auto wait = [&](uint64_t* b, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, wait_ns));
+    };
+    int entries = 0, last_q = -1, pending = -1;
+    bool ok = true;
+    for (int pc = 0; pc < npieces && ok; ++pc) {
+      const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+      if (lane == 0 && p.seqlens[pz.seq] > p.bt_stride * kPage)
+        report(p.status, MLA_ERR_DEVICE_CHECK);
+      if (pz.npg == 0) continue;
+      const int cnt = p.seqlens[pz.seq];
+      const int32_t* grows = p.gather_rows + static_cast<int64_t>(pz.seq) * p.gather_stride;
+      auto rows_of = [&](int jj, int (&r)[2]) {  // this lane's rows: lane and lane + 32
+        const int vt0 = (pz.pg0 + jj) * kPage;
+        for (int h = 0; h < 2; ++h) {
+          const int tok = vt0 + 32 * h + lane;
+          r[h] = tok < cnt ? __ldg(grows + tok) : -1;  // past the count: a zero row
+        }
+      };
+      int next[2];
+      rows_of(0, next);
+      for (int e = -1; e < pz.npg; ++e) {  // e = -1: the query rows
+        const int stage = entries % kStages, use = entries / kStages;
+        if (use > 0) {
+          ok = wait(&bar[kEmpty0 + stage], (use - 1) & 1);
+          if (!ok) break;
+        }
+        uint8_t* dst = skv + stage * kTileBytes;
+        if (e < 0) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[kFull0 + stage], kTileBytes);
+            const int qrow = pz.seq * p.rows + rb * kRowsPerCta;
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_q, c * 64, qrow, &bar[kFull0 + stage]);
+          }
+          last_q = entries;
+        } else {
+          const int mine[2] = {next[0], next[1]};
+          if (e + 1 < pz.npg) rows_of(e + 1, next);
+          const int u = lane & 7;
+#pragma unroll
+          for (int grp = 0; grp < 16; ++grp) {
+            const int r = 4 * grp + (lane >> 3);
+            const int row = __shfl_sync(0xffffffffu, grp < 8 ? mine[0] : mine[1], r & 31);
+            const uint8_t* src = static_cast<const uint8_t*>(p.gather_cache) +
+                                 static_cast<int64_t>(row < 0 ? 0 : row) * (kDqk * 2) + u * 16;
+            uint8_t* d = dst + r * 128 + ((u ^ (r & 7)) << 4);
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+              cp_async16_zfill(d + c * kChunkBytes, src + c * 128, row >= 0);
+          }
+          cp_async_commit();
+          if (pending >= 0) {
+            cp_async_wait_group<1>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kFull0 + pending]);
+          }
+          pending = stage;
+          if (e + 1 == pz.npg) {  // the piece's last page: signal it now
+            cp_async_wait_group<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kFull0 + pending]);
+            pending = -1;
+          }
+        }
+        ++entries;
+      }
+    }
+    // Before leaving, let every copy this warp issued land (bounded): the page
+    // copies, and the last query load if no later entry reused its stage.
+    cp_async_wait_group<0>();
+    if (lane == 0 && last_q >= 0 && last_q >= entries - kStages)
+      mbar_wait_drain(&bar[kFull0 + last_q % kStages], (last_q / kStages) & 1, kWaitLimitNs);
   } else if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -710,6 +796,9 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
     e = cudaFuncSetAttribute(mla_decode_sm100_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemBytes);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(mla_decode_sm100_kernel<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemBytes);
+    if (e != cudaSuccess) return e;
     configured[dev].store(true, std::memory_order_release);
   }
   const int row_blocks = (p.rows + kRowsPerCta - 1) / kRowsPerCta;
@@ -723,7 +812,10 @@ cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel<false>, tm_q, tm_page, p);
+  if (p.gather_rows != nullptr)
+    e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel<false, true>, tm_q, tm_page, p);
+  else
+    e = cudaLaunchKernelEx(&cfg, mla_decode_sm100_kernel<false>, tm_q, tm_page, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -40,6 +40,12 @@ struct DecodeParams {
                         // through mla_set_wait_limit_ns)
   const int32_t* stall_flag;  // test hook, normally null: when set, the PV issuer waits
                               // for it to become non-zero before its first PV
+  // Gathered rows (sparse decode on CTA pairs): token k of sequence s is cached
+  // row gather_rows[s * gather_stride + k] of gather_cache [rows, 576] bf16;
+  // null for the dense decode, which reads pages through the block table.
+  const int32_t* gather_rows;
+  const void* gather_cache;
+  int64_t gather_stride;
 };
 
 struct CombineParams {
@@ -81,19 +87,17 @@ struct ReleaseParams {
   int batch, free_capacity;
 };
 
-// Sparse decode: compaction of used indices and gather of their rows (mla_sparse.cu).
+// Sparse decode: compaction of the used index entries into cached rows (mla_sparse.cu).
 struct SparseParams {
   const int32_t* indices;      // [batch * s_q, topk]
   const int32_t* seqlens;      // [batch]
   const int32_t* block_table;  // [batch, bt_stride]
-  const void* kcache;          // [num_blocks * 64, 576] bf16
-  int32_t* comp;               // workspace [batch * s_q, topk]: used entries, in order
+  int32_t* comp;               // workspace [batch * s_q, topk]: cached rows of the used
+                               // entries, in list order
   int32_t* counts;             // workspace [batch * s_q]
-  int32_t* comp_bt;            // workspace [batch * s_q, pages_per_pos]
-  void* comp_cache;            // workspace [batch * s_q * pages_per_pos * 64, 576] bf16
   int32_t* status;             // nullable
   int64_t bt_stride, num_blocks;
-  int batch, s_q, topk, causal, pages_per_pos;
+  int batch, s_q, topk, causal;
 };
 
 // Launchers (return cudaGetLastError() of their launch).
@@ -112,6 +116,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
+// With p.gather_rows set, the K and V parts are copied row by row from
+// p.gather_cache (tm_kpart and tm_vx are not read).
 cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
                                const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
                                const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,

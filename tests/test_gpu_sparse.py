@@ -81,3 +81,47 @@ def test_sparse_full_list_equals_dense(cuda_device):
     dense = run_cuda(inp, cuda_device)
     np.testing.assert_allclose(out, dense["out"], atol=1e-2, rtol=1e-2)
     np.testing.assert_allclose(lse, dense["lse"], atol=1e-3)
+
+
+@pytest.mark.parametrize("s_q,causal", [(1, False), (2, True)])
+def test_sparse_full_list_equals_dense_on_pairs(cuda_device, s_q, causal):
+    # 128 heads: the pair kernel copies the listed rows itself; with every
+    # position listed, in order, it must agree with the dense decode
+    from parity import run_cuda
+    w = synth.custom_workload(3, s_q, 128, [130, 64, 1000], causal=causal)
+    inp = synth.make_inputs(w, seed=78 + s_q)
+    idx = torch.full((3, s_q, 1000), -1, dtype=torch.int32)
+    for i, L in enumerate(inp.cache_seqlens.tolist()):
+        idx[i, :, :L] = torch.arange(L, dtype=torch.int32)
+    out, lse = run_sparse(inp, idx, cuda_device)
+    dense = run_cuda(inp, cuda_device)
+    np.testing.assert_allclose(out, dense["out"], atol=1e-2, rtol=1e-2)
+    np.testing.assert_allclose(lse, dense["lse"], atol=1e-3)
+
+
+@pytest.mark.parametrize("h_q", [16, 128])
+def test_sparse_entry_on_a_page_outside_the_cache(cuda_device, h_q):
+    # a used entry whose block-table page lies outside the cache is read as a
+    # zero row and reported; the rest of the result is exact
+    from mla_paged_latent_decode_b200 import binding
+    w = synth.custom_workload(2, 1, h_q, [300, 200])
+    inp = synth.make_inputs(w, seed=79)
+    nb = inp.kcache.shape[0]
+    idx = synth.make_sparse_indices(inp, 40, seed=79)
+    idx[0, 0, 0] = 70                      # token 70 lives in logical page 1 of sequence 0
+    bad_bt = inp.block_table.clone()
+    bad_bt[0, 1] = nb + 5                  # ... which now points past the cache
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out, lse = binding.mla_decode_sparse(inp.q.to(cuda_device), inp.kcache.to(cuda_device),
+                                         bad_bt.to(cuda_device), inp.cache_seqlens.to(cuda_device),
+                                         idx.to(cuda_device), inp.scale, False,
+                                         device_status=status)
+    torch.cuda.synchronize(cuda_device)
+    assert int(status.item()) == binding.MLA_ERR_DEVICE_CHECK
+    # the oracle on a cache with one more page, all zeros, in place of the bad one
+    kc = torch.cat([inp.kcache, torch.zeros((1, 64, 576), dtype=torch.bfloat16)])
+    zero_bt = inp.block_table.clone()
+    zero_bt[0, 1] = nb
+    ref_out, ref_lse = sparse.decode(inp.q, kc, zero_bt, inp.cache_seqlens, idx, inp.scale, False)
+    assert_close_out(out.float().cpu().numpy(), ref_out, "sparse out")
+    assert_close_lse(lse.cpu().numpy(), ref_lse, "sparse lse")
