@@ -366,7 +366,7 @@ def measure_workload(name, dev, stream, flush_l2, reps, peaks):
     kernel = "pair" if s_q * h_q > 64 else "single-CTA"
     return {
         "workload": f"{name}: {inp.workload.description}", "kernel": kernel, "num_workers": nw,
-        "pieces": None, "bytes": nbytes, "flops": flops,
+        "bytes": nbytes, "flops": flops,
         "decode_call_us": call_us[0], "decode_call_us_p10": call_us[1],
         "decode_call_us_p90": call_us[2],
         "step_us": step_us[0], "step_us_p10": step_us[1], "step_us_p90": step_us[2],
