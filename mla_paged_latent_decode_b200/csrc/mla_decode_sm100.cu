@@ -36,7 +36,7 @@
 // FP8 cache (template argument kFp8): the same kernel over E4M3 codes with one
 // power-of-two scale per token.  The TMA warp lands each page chunk's codes in
 // the upper half of that chunk's 128-byte row slots inside the bf16 stage, and
-// four more warps (384 threads) widen them in place into the bf16 tile, exactly;
+// eight more warps (512 threads) widen them in place into the bf16 tile, exactly;
 // the MMAs, softmax and epilogue are unchanged.
 //
 // The method follows "FlashMLA: Revolutionizing Efficient Decoding...",
@@ -60,8 +60,9 @@ constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;    // issues QK^T of even pages; allocates tensor memory
 constexpr int kPvWarp = 6;     // issues PV
 constexpr int kQkOddWarp = 7;  // issues QK^T of odd pages
-constexpr int kConvWarp0 = 8;  // FP8 cache: first of four converter warps
-constexpr int kConvThreads = 128;
+constexpr int kConvWarp0 = 8;  // FP8 cache: first of eight converter warps
+constexpr int kConvThreads = 256;
+constexpr int kConvChunkStep = kConvThreads / 64;  // chunks apart of one thread's row slots
 constexpr int kConvBarrier = 1;                    // named barrier of the converter warps
 constexpr int kChunkBytes = 64 * 128;              // 64 rows x 64 bf16 (one swizzle column block)
 constexpr int kChunks = kDqk / 64;                 // 9
@@ -204,9 +205,10 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // FP8 cache: 384 threads launched with 168 registers each; the softmax
+  // FP8 cache: 512 threads launched with 128 registers each; the softmax
   // warpgroup raises its budget to 232, the single-thread roles (warps 4-7)
-  // lower theirs to 56 and the converters to 128: 53248 of the 64512 in all.
+  // lower theirs to 56 and the two converter warpgroups to 96: 61440 of the
+  // 65536 in all.
   if constexpr (kFp8) {
     if (warp >= 4 && warp < kConvWarp0) setmaxnreg_dec<56>();
   }
@@ -278,16 +280,16 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (kFp8 && warp >= kConvWarp0) {
     // ------------------------------------------------------------ FP8 converters
     // Widen each landed page in place: thread t owns row r = t % 64 of chunks
-    // t / 64, t / 64 + 2, ... (5 or 4 of the 9).  For each it reads the 64
+    // t / 64, t / 64 + 4, ... (3 or 2 of the 9).  For each it reads the 64
     // codes (bytes 64..127 of the row slot) into registers, then writes the 64
     // bf16 values over the whole 128-byte slot, swizzled.  No other thread
     // touches that slot, so reading before writing makes the in-place update
     // safe.  The four 16-byte loads start at unit (r mod 4) and the eight 8-lane
     // store phases cover 8 rows, so neither hits a bank more than twice.  Rows
     // past the sequence's end are written as zeros, so stale codes or scales
-    // there never reach an MMA.  The four warps decide together after a named
+    // there never reach an MMA.  The eight warps decide together after a named
     // barrier, so that a wait that gave up in one warp stops all of them.
-    if constexpr (kFp8) setmaxnreg_dec<128>();
+    if constexpr (kFp8) setmaxnreg_dec<96>();
     const int ct = threadIdx.x - kConvWarp0 * 32;
     const int r = ct & 63, c0 = ct >> 6;
     int entries = 0;
@@ -312,7 +314,7 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                            0x10001u
                                      : 0u;
         constexpr uint32_t f_hi = 0x5D805D80u;  // 2^60 in both halves
-        for (int c = c0; c < kChunks; c += 2) {
+        for (int c = c0; c < kChunks; c += kConvChunkStep) {
           uint8_t* slot = tile + c * kChunkBytes + r * 128;
           uint4 v[4];
 #pragma unroll

@@ -217,3 +217,15 @@ def test_overlong_sequence_is_reported_not_read(cuda_device):
     res = run_cuda(inp, cuda_device)
     from mla_paged_latent_decode_b200 import binding
     assert res["status"] == binding.MLA_ERR_DEVICE_CHECK
+
+
+@pytest.mark.parametrize("h_q", [16, 128])
+def test_large_batch_of_short_sequences(cuda_device, h_q):
+    # many more sequences than workers: every worker runs many pieces, the
+    # scheduler's worker rows span thousands of sequences
+    g = torch.Generator().manual_seed(5)
+    b = 3000 if h_q == 16 else 600
+    lens = torch.randint(0, 300, (b,), generator=g).tolist()
+    w = synth.custom_workload(b, 1, h_q, lens)
+    inp = synth.make_inputs(w, seed=81)
+    full_parity(inp, cuda_device)
