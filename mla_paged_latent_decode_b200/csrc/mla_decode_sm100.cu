@@ -4,9 +4,11 @@
 // worker's run of (sequence, page) items (see mla_metadata.cu).
 //
 // Data movement and math per page:
-//   TMA   : the 64 x 576 bf16 page (72 KB) -> shared memory as 9 boxes of
-//           64 x 64 with 128-byte swizzle, through the block table; a ring of
-//           three stages.  At the start of each piece the same ring also
+//   TMA   : the 64 x 576 bf16 page (72 KB) -> shared memory as one 3-D box
+//           (nine 64-dim chunks of 64 rows) with 128-byte swizzle, through the
+//           block table; a ring of three stages.  In gather mode (sparse
+//           decode) the producer warp's lanes copy the page's listed rows
+//           instead, with 16-byte cp.async copies into the same layout.  At the start of each piece the same ring also
 //           carries the piece's 64 query rows (72 KB), which the softmax warps
 //           move into tensor memory.
 //   MMA   : S  = Q . K^T    tcgen05 M=64 N=64 K=576, A = Q in TMEM, B = page

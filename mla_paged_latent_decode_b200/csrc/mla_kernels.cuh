@@ -108,11 +108,15 @@ cudaError_t launch_append(const AppendParams& p, bool fp8, cudaStream_t stream);
 cudaError_t launch_release(const ReleaseParams& p, cudaStream_t stream);
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, int piece_cost,
                             int32_t* tile_md, int32_t* num_splits, cudaStream_t stream);
+// Single-CTA kernel (up to 64 query rows per sequence; more rows run as several
+// 64-row blocks).  With p.gather_rows set, each page's rows are copied by index
+// from p.gather_cache (tm_page is not read).
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
-// FP8 (E4M3) cache, up to 64 query rows per sequence: tm_page8 views the codes
-// as [rows, 576] bytes in boxes of 128 bytes x 64 rows; scales via p.kscale.
+// FP8 (E4M3) cache, any number of query rows (one CTA per worker and 64-row
+// block): tm_page8 views the codes as [rows, 576] bytes in boxes of 128 bytes x
+// 64 rows; scales via p.kscale.
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
