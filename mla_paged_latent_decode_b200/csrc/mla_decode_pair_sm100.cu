@@ -263,22 +263,16 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
-  // Launched as a programmatic dependent of the scheduler kernel: its CTAs may
-  // start while the scheduler runs, and read the metadata only after this wait.
-  grid_dependency_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int worker = blockIdx.x >> 1, rb2 = blockIdx.y;
-  const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
-  const int npieces = md[5];
-  if (npieces == 0) return;  // idle worker: both CTAs of the pair leave together
-  if (md[0] < 0 || npieces < 0 || md[0] + npieces > p.batch) {
-    if (threadIdx.x == 0 && rank == 0) report(p.status, MLA_ERR_DEVICE_CHECK);
-    return;
-  }
   const int row0 = rb2 * 128 + 64 * static_cast<int>(rank);  // first query row of this CTA
   const uint64_t wait_ns = p.wait_ns;  // limit of every bounded wait (normally kWaitLimitNs)
 
+  // Set-up first: the kernel is launched as a programmatic dependent of the
+  // scheduler kernel, so its CTAs may start while the scheduler runs; barriers
+  // and tensor memory are made ready meanwhile, and the metadata is read only
+  // after the dependency wait below.
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&bar[kKFull0 + s], kFullArrivals);
@@ -310,11 +304,26 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();
   }
+  if (warp == kTmaKWarp && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    if (!kGather) prefetch_tensormap(&tm_kpart);
+  }
+  if (warp == kTmaVWarp && lane == 0 && !kGather) prefetch_tensormap(&tm_vx);
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // barriers and tensor memory of both CTAs exist before either uses them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  grid_dependency_wait();  // the scheduler's metadata is complete and visible
+  const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
+  int npieces = md[5];
+  if (npieces != 0 && (md[0] < 0 || npieces < 0 || md[0] + npieces > p.batch)) {
+    if (threadIdx.x == 0 && rank == 0) report(p.status, MLA_ERR_DEVICE_CHECK);
+    npieces = 0;
+  }
+  // An idle worker (or bad metadata) runs no role: both CTAs of the pair read
+  // the same row and go straight to the common teardown.
 
   // Every role walks the same sequence of K-ring entries: per piece with pages,
   // two query-staging entries, then one entry per page.
@@ -325,10 +334,6 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // page is signalled once two newer pages have been issued (up to three
     // pages of copies in flight), a piece's last pages at the piece's end.
     if (kGather || lane == 0) {
-      if (lane == 0) {
-        prefetch_tensormap(&tm_q);
-        if (!kGather) prefetch_tensormap(&tm_kpart);
-      }
       // a wait of the lanes running this loop, with the same outcome in each
       auto wait = [&](uint64_t* b, uint32_t parity) {
         bool r = mbar_wait_cluster(b, parity, abort_flag, wait_ns);
@@ -339,6 +344,14 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       int pending[2] = {-1, -1};  // gather: slots of the two newest pages not yet signalled
       bool ok = true;
       for (int pc = 0; pc < npieces && ok; ++pc) {
+        // dense pages: the block-table entry of the piece's first page, loaded
+        // together with the piece's length (both follow from the metadata alone)
+        const int32_t* bt = p.block_table + static_cast<int64_t>(md[0] + pc) * p.bt_stride;
+        int page_next = 0;
+        if constexpr (!kGather) {
+          const int pg0 = pc == 0 ? md[1] : 0;
+          page_next = __ldg(bt + (pg0 >= 0 && pg0 < p.bt_stride ? pg0 : 0));
+        }
         const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
         if (lane == 0 && rank == 0 && p.seqlens[pz.seq] > p.bt_stride * kPage)
           report(p.status, MLA_ERR_DEVICE_CHECK);
@@ -415,8 +428,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
               pending[0] = pending[1] = -1;
             }
           } else {
-            const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
-            const int page = __ldg(bt + pz.pg0 + j);
+            // this page's entry was loaded one page ahead; load the next one
+            // before waiting for the slot
+            const int page = page_next;
+            if (j + 1 < pz.npg) page_next = __ldg(bt + pz.pg0 + j + 1);
             if (use > 0) {
               ok = wait(&bar[kKEmpty0 + slot], (use - 1) & 1);
               if (!ok) break;
@@ -445,7 +460,6 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // Dense pages: one TMA box (lane 0).  Gathered rows: all lanes copy the
     // peer tokens' rows and signal the page once their copies have landed.
     if (kGather || lane == 0) {
-      if (!kGather) prefetch_tensormap(&tm_vx);
       const int xgrp = rank == 0 ? 1 : 0;
       const int dst_chunk = rank == 0 ? kXChunks : 0;
       const int src_row = rank == 0 ? 32 : 0, src_chunk = rank == 0 ? 0 : kXChunks;
@@ -729,8 +743,9 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       // ---- epilogue: sums of the two row halves, then O / l.  Each warp owns
       // rows 32 (warp & 1) .. +31 of this CTA and dv half `th` of each 256-wide
       // block.  Blocks go TMEM -> registers -> shared memory (the P buffers,
-      // idle until this piece's output is written; 16-byte units XOR-swizzled by
-      // row, so neither side has bank conflicts) -> global memory: by TMA store
+      // idle until this piece's output is written, or the idle ring after the
+      // CTA's last piece; 16-byte units XOR-swizzled by row, so neither side has
+      // bank conflicts) -> global memory: by TMA store
       // for fp32 partials and for the bf16 output of the CTA's last piece, by
       // the load/store units (one contiguous row segment per instruction) for
       // the bf16 output of an earlier piece.
@@ -743,14 +758,22 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       float* stg = reinterpret_cast<float*>(sp) + warp * 1024;
       const int wrow0 = row0 + 32 * (warp & 1);  // sequence row of this warp's lane 0
+      // The dependent grid (the split combine) may be scheduled once every CTA
+      // has reached its last epilogue; it still waits for this grid's end
+      // before it reads anything, and a step without splits ends it at once.
+      if (pc == npieces - 1 && threadIdx.x == 0) grid_launch_dependents();
       if (k_pieces == 1 && pc == npieces - 1) {
         // bf16 output of this CTA's last piece: blocks of 32 rows x 64 dv columns
         // (128 bytes per row), one TMA store each (rows past the sequence's query
         // rows fall outside the map and are not written).  Only the last piece:
-        // earlier, TMA stores would queue with the next piece's page loads.
+        // earlier, TMA stores would queue with the next piece's page loads.  The
+        // ring is idle by now (every load landed and every MMA that read it is
+        // done), so each block gets its own 4 KB staging buffer there and the
+        // four stores of a warp go out back to back.
         for (int h = 0; h < 2; ++h) {
           for (int cb = 0; cb < 128; cb += 64) {
             const int col = 128 * h + 256 * th + cb;
+            float* stg_blk = reinterpret_cast<float*>(sk) + (warp * 4 + 2 * h + cb / 64) * 1024;
             uint32_t w[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -767,19 +790,16 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 w[16 * half + k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv,
                                                __uint_as_float(o[2 * k + 1]) * inv);
             }
-            // the TMA store of the previous block has read the staging buffer
-            if (lane == 0) tma_store_wait_read();
-            __syncwarp();
             // row `lane` -> 16-byte unit u ^ (lane & 7) of staging row `lane` (the
             // layout of a 128-byte-swizzled TMA box of 32 rows x 64 bf16)
-            uint4* srow = reinterpret_cast<uint4*>(stg + lane * 32);
+            uint4* srow = reinterpret_cast<uint4*>(stg_blk + lane * 32);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
               srow[u ^ (lane & 7)] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&tm_out, stg, col, wrow0, pz.seq);
+              tma_store_3d(&tm_out, stg_blk, col, wrow0, pz.seq);
               tma_store_commit();
             }
             __syncwarp();
@@ -856,7 +876,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   }
 
-  if (warp < kSoftmaxWarps && lane == 0) tma_store_wait_all();  // partial outputs written
+  // The stores have read their staging buffers before the CTA exits; their
+  // writes complete with the grid (the combine kernel and the host see them
+  // after its end).
+  if (warp < kSoftmaxWarps && lane == 0) tma_store_wait_read();
   // After an abort, work this CTA issued may still be in flight: pair MMAs of the
   // leader's issuing threads (each waits for its own to complete, through a
   // commit), and TMA loads of either CTA (they cannot be cancelled and land

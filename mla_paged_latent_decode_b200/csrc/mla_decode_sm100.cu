@@ -715,6 +715,10 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!ok) break;
         tc_fence_after();
       }
+      // The dependent grid (the split combine) may be scheduled once every CTA
+      // has reached its last epilogue; it still waits for this grid's end
+      // before it reads anything.
+      if (pc == npieces - 1 && threadIdx.x == 0) grid_launch_dependents();
       // ---- epilogue: the four threads of a row group hold disjoint columns
       l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
       l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
