@@ -272,16 +272,17 @@ int mla_append_latent_fp8(const void* rows, int s_new, void* kcache, float* ksca
  *
  * kcache:  device uint8 [num_blocks, 64, 576] E4M3 codes, 16-byte aligned.
  * kscale:  device fp32 [num_blocks, 64] per-token scales, 16-byte aligned.
- * Rows of a sequence's last page past its length are never read as data (the
- * kernel zeroes them), so their codes and scales may hold anything.  Widening
- * is exact for scales 2^k with -124 <= k <= 67 (what the quantising append
- * writes for rows whose largest magnitude lies in about [1e-35, 6.6e22]).
- * Any s_q * h_q up to 65536 (MLA_ERR_UNSUPPORTED above): one CTA per worker
- * and 64-row block of query rows (the blocks of one worker run side by side and
- * read the same pages, the second time mostly from L2); metadata from
- * mla_get_metadata as for mla_decode_kvcache (with more than 64 rows its
- * worker count keeps every CTA of the grid resident at once).  All other
- * arguments, the workspace, errors and launches are as for mla_decode_kvcache.
+ * Rows of a sequence's last page past its length are never read as data
+ * (zeroed, or masked with zero probability), so their codes and scales may
+ * hold anything.  Widening is exact for scales 2^k with -124 <= k <= 67 (what
+ * the quantising append writes for rows whose largest magnitude lies in about
+ * [1e-35, 6.6e22]).  Any s_q * h_q up to 65536 (MLA_ERR_UNSUPPORTED above):
+ * up to 64 query rows per sequence on single CTAs (codes widened to code *
+ * scale), more on CTA pairs like mla_decode_kvcache (codes widened to their
+ * values, each token's scale applied to its score and, exactly, to its
+ * probability).  Metadata from mla_get_metadata as for mla_decode_kvcache.
+ * All other arguments, the workspace, errors and launches are as for
+ * mla_decode_kvcache.
  */
 int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscale,
                            int64_t num_blocks, const int32_t* block_table, int bt_stride,

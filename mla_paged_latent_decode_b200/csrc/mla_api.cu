@@ -134,6 +134,27 @@ bool make_fp8_page_map(CUtensorMap* map, const void* base, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
+// The E4M3 cache viewed as 3-D {128 bytes, rows, 9 chunks} with strides of 576
+// bytes (a row) and 64 bytes (a chunk): element (x, r, c) is byte 64 c + x of
+// row r.  A box of 128 x box_rows x box_chunks started at x = -64 lands, for
+// each chunk, 64 zero bytes (x < 0 is out of bounds) and then the chunk's 64
+// codes in each 128-byte row slot, chunk after chunk: the layout the pair
+// kernel's converters widen, in one TMA instruction.  (x never reaches 64, so
+// no element past a row is read.)
+bool make_fp8_chunk_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows,
+                        uint32_t box_chunks) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(mla::kDqk / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk), 64};
+  cuuint32_t box[3] = {128, box_rows, box_chunks};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Query rows up to 64 per sequence run on single CTAs (one 64-row block); more
@@ -373,10 +394,18 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   if (need == 0 || workspace_bytes < need) return MLA_ERR_INVALID_ARG;
 
   const int rows = s_q * h_q;
-  CUtensorMap tm_q, tm_page8;
+  const bool pairs = uses_pairs(s_q, h_q);
+  const uint64_t cache_rows = static_cast<uint64_t>(num_blocks) * mla::kPage;
+  CUtensorMap tm_q, tm_page8 = {}, tm_k8 = {}, tm_v8 = {};
   if (!make_row_map(&tm_q, q, static_cast<uint64_t>(batch) * rows)) return MLA_ERR_CUDA;
-  if (!make_fp8_page_map(&tm_page8, kcache, static_cast<uint64_t>(num_blocks) * mla::kPage))
+  if (pairs) {
+    // a CTA of a pair: its 32 tokens x 9 chunks, or 32 tokens x 4 chunks of values
+    if (!make_fp8_chunk_map(&tm_k8, kcache, cache_rows, 32, mla::kDqk / 64) ||
+        !make_fp8_chunk_map(&tm_v8, kcache, cache_rows, 32, 4))
+      return MLA_ERR_CUDA;
+  } else if (!make_fp8_page_map(&tm_page8, kcache, cache_rows)) {
     return MLA_ERR_CUDA;
+  }
   const size_t slots = static_cast<size_t>(batch) + static_cast<size_t>(num_workers);
   float* part_o = static_cast<float*>(workspace);
   float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -403,8 +432,17 @@ int mla_decode_kvcache_fp8(const void* q, const void* kcache, const float* kscal
   p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   p.stall_flag = g_stall_flag.load(std::memory_order_relaxed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (mla::launch_decode_fp8(tm_q, tm_page8, p, num_workers, st) != cudaSuccess)
+  if (pairs) {
+    CUtensorMap tm_po, tm_out;
+    if (!make_partial_map(&tm_po, part_o, static_cast<uint64_t>(rows), slots)) return MLA_ERR_CUDA;
+    if (!make_out_map(&tm_out, out, static_cast<uint64_t>(rows), static_cast<uint64_t>(batch)))
+      return MLA_ERR_CUDA;
+    if (mla::launch_decode_pair_fp8(tm_q, tm_k8, tm_v8, tm_po, tm_out, p, num_workers, st) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
+  } else if (mla::launch_decode_fp8(tm_q, tm_page8, p, num_workers, st) != cudaSuccess) {
     return MLA_ERR_CUDA;
+  }
   return launch_combine_for(num_splits, part_o, part_lse, out, lse, batch, s_q, h_q, rows, st);
 }
 

@@ -59,6 +59,18 @@
 // P is double-buffered, so the softmax of page g overlaps PV of page g - 1; the
 // softmax waits for that PV only when it has to rescale O.
 //
+// FP8 cache (template argument kFp8, 640 threads): E4M3 codes with one
+// power-of-two scale per token.  The same slots, MMAs and barriers, with the
+// loads and their completion changed: one TMA box per K part lands each
+// chunk's codes in the upper half of its 128-byte row slots (a view of the
+// codes whose chunks are 64 bytes apart, started 64 bytes early), and the
+// page's 64 scales come with it; two groups of four converter warps (even and
+// odd pages) widen the codes in place to bf16 values equal to the codes, and
+// three more warps widen the peer tokens' value chunks the value warp loads the
+// same way.  Each group signals the leader's barrier once per CTA.  The scales
+// are applied in the softmax: to each token's score, and to its probability
+// before P goes to PV (a power of two: exact in bf16).
+//
 // The method is that of the single-CTA kernel ("FlashMLA: Revolutionizing
 // Efficient Decoding...", sections 4.2.1-4.2.3: TMA prefetch of 64-row latent
 // blocks, tensor cores for QK^T and PV, softmax fused in the kernel), mapped
@@ -71,13 +83,38 @@
 namespace mla {
 namespace {
 
-constexpr int kThreads = 288;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kTmaKWarp = 4;
 constexpr int kQkEvenWarp = 5;
 constexpr int kPvWarp = 6;
 constexpr int kQkOddWarp = 7;
-constexpr int kTmaVWarp = 8;
+// Threads and the warp of the value loads: 288 threads (warp 8 loads values)
+// for a bf16 cache.  For an FP8 cache, 640: two groups of four warps (8-11 and
+// 12-15) widen the K parts of even and odd pages, warp 16 loads values and
+// warps 17-19 widen them.
+template <bool kFp8>
+struct PairRoles {
+  static constexpr int kThreads = kFp8 ? 640 : 288;
+  static constexpr int kTmaVWarp = kFp8 ? 16 : 8;
+};
+constexpr int kKConvWarp0 = 8;                 // FP8: K-part converters, warps 8..15
+constexpr int kKConvGroups = 2;                // of four warps each, alternating pages
+constexpr int kKConvThreads = 128;             // per group
+constexpr int kVConvWarp0 = 17;                // FP8: value converters, warps 17..19
+constexpr int kVConvThreads = 96;
+constexpr int kVConvBarrier = 1;               // named barriers: the value converters,
+constexpr int kKConvBarrier0 = 2;              //   then one per K-converter group
+// FP8 register budget: 640 threads are launched with at most 102 registers
+// each (the launcher checks kFp8LaunchRegs); the converter warpgroups lower
+// theirs and the softmax warpgroup raises its own.
+constexpr int kFp8LaunchRegs = 96;
+constexpr int kFp8RegsSoftmax = 176, kFp8RegsConv = 64;
+static_assert(128 * kFp8RegsSoftmax + 128 * kFp8LaunchRegs + 384 * kFp8RegsConv <=
+                  640 * kFp8LaunchRegs,
+              "FP8 setmaxnreg split within the launch's registers");
+// bf16 2^120: widened codes are code * 2^120 * 2^-120 = the code itself; each
+// token's scale is applied to its scores and probabilities instead
+constexpr uint32_t kBf16x2Pow120 = 0x7B807B80u;
 
 constexpr int kChunk = 64 * 128;          // 64 rows x 64 bf16 (one 128-byte swizzle column block)
 constexpr int kHalfChunk = 32 * 128;      // 32 rows x 64 bf16
@@ -104,7 +141,9 @@ constexpr int kOffK = kOffQ2 + kQ2Bytes;
 constexpr int kOffP = kOffK + kKSlots * kKBytes;
 constexpr int kOffX = kOffP + 2 * kPBytes;       // row-half exchange: [2 pages][2 halves][64] f32
 constexpr int kOffL = kOffX + 2 * 2 * 64 * 4;    // epilogue sum exchange: [2 pieces][2 halves][64] f32
-constexpr int kOffBar = kOffL + 2 * 2 * 64 * 4;
+constexpr int kOffScale = kOffL + 2 * 2 * 64 * 4;  // FP8: [slot][64] fp32: this CTA's 32
+                                                    // tokens, then the 32 peer tokens' values
+constexpr int kOffBar = kOffScale + kKSlots * kPage * 4;
 static_assert(kOffK % 1024 == 0 && kKBytes % 1024 == 0 && kOffP % 1024 == 0,
               "swizzled tiles start on 1024-byte boundaries");
 enum Bar {
@@ -123,7 +162,9 @@ enum Bar {
   kXBar, kLBar,                                   // local: softmax exchanges
   kDrain0,                                        // leader: MMA drain after an abort, one
                                                   //   per issuing warp (5, 6, 7)
-  kNumBars = kDrain0 + 3
+  kKLanded0 = kDrain0 + 3,                        // FP8, local: a K part's codes and scales
+  kVLanded0 = kKLanded0 + kKSlots,                // FP8, local: values' codes and scales
+  kNumBars = kVLanded0 + kKSlots
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffMisc + 16;
@@ -218,6 +259,57 @@ __device__ __forceinline__ bool copy_query_rows(const uint8_t* sk, uint64_t* bar
   return true;
 }
 
+// FP8 converters: wait for a landed barrier (bounded), then decide together
+// after a named barrier, so that a wait that gave up in one warp (it raises the
+// abort flag) stops all of them.  Returns false to stop.
+__device__ __forceinline__ bool convert_wait(uint64_t* landed, uint32_t parity,
+                                             volatile int* abort_flag, uint64_t wait_ns,
+                                             int named_barrier, int threads) {
+  mbar_wait(landed, parity, abort_flag, wait_ns);
+  named_bar_sync(named_barrier, threads);
+  return *abort_flag == 0;
+}
+
+// Widen one 128-byte row slot in place: its 64 E4M3 codes (bytes 64..127, as
+// the TMA box landed them) become the 64 codes as bf16 values over the whole
+// slot, in the 128-byte-swizzled layout (16-byte unit u of row r at (u ^ (r %
+// 8)) * 16).  For a code b = s eeee mmm the 16-bit pattern s 0000 eeee mmm 0000
+// is the bf16 value b * 2^-120 (E4M3 subnormals become bf16 subnormals); one
+// bf16x2 multiply by 2^120 makes it b, exactly.  A pattern is never NaN or
+// infinite, so rows past a sequence's end hold finite values (their scores are
+// masked and their probabilities are zero).  The four 16-byte loads start at
+// unit (r mod 4), so the lanes of a warp spread over the banks.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_codes(uint32_t word, uint32_t sel) {
+  const uint32_t t = __byte_perm(word, 0u, sel);  // (b_hi << 24) | (b_lo << 8)
+  const uint32_t pat = ((t & 0x7F007F00u) >> 4) | (t & 0x80008000u);
+  const uint32_t f = kBf16x2Pow120;
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pat);
+  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void widen_row_slot(uint8_t* slot, int r) {
+  uint4 v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    v[k] = *reinterpret_cast<const uint4*>(slot + 64 + 16 * ((k + r) & 3));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int kk = (k + r) & 3;  // v[k] holds dims 16 kk .. 16 kk + 15 of the chunk
+    uint4 lo, hi;
+    lo.x = e4m3x2_to_bf16x2_codes(v[k].x, 0x1404u);
+    lo.y = e4m3x2_to_bf16x2_codes(v[k].x, 0x3424u);
+    lo.z = e4m3x2_to_bf16x2_codes(v[k].y, 0x1404u);
+    lo.w = e4m3x2_to_bf16x2_codes(v[k].y, 0x3424u);
+    hi.x = e4m3x2_to_bf16x2_codes(v[k].z, 0x1404u);
+    hi.y = e4m3x2_to_bf16x2_codes(v[k].z, 0x3424u);
+    hi.z = e4m3x2_to_bf16x2_codes(v[k].w, 0x1404u);
+    hi.w = e4m3x2_to_bf16x2_codes(v[k].w, 0x3424u);
+    *reinterpret_cast<uint4*>(slot + (((2 * kk) ^ (r & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(slot + (((2 * kk + 1) ^ (r & 7)) << 4)) = hi;
+  }
+}
+
 // Gathered rows: copy 32 cached rows (this lane holds the row index of row
 // `lane`; -1 = a zero row) into a slot, chunks src_chunk .. src_chunk +
 // nchunks - 1 of each row to chunks dst_chunk .. of the slot, in the
@@ -241,8 +333,8 @@ __device__ __forceinline__ void gather_rows32(uint8_t* slot, int dst_chunk, int 
   }
 }
 
-template <bool kGather>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kGather, bool kFp8>
+__global__ void __launch_bounds__(PairRoles<kFp8>::kThreads, 1)
 mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kpart,
                        const __grid_constant__ CUtensorMap tm_vx,
@@ -251,14 +343,20 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // full barriers of the K and V parts: one TMA-counted arrival (dense pages),
-  // or one arrival per CTA (gathered rows, copied by the threads)
-  constexpr uint32_t kFullArrivals = kGather ? 2 : 1;
+  static_assert(!(kGather && kFp8), "gathered rows come from a bf16 cache");
+  constexpr int kThreads = PairRoles<kFp8>::kThreads;
+  constexpr int kTmaVWarp = PairRoles<kFp8>::kTmaVWarp;
+  // full barriers of the K and V parts: one TMA-counted arrival (dense bf16
+  // pages), or one arrival per CTA (gathered rows, copied by the threads; FP8
+  // codes, widened by the converter warps)
+  constexpr uint32_t kFullArrivals = (kGather || kFp8) ? 2 : 1;
+  (void)kThreads;
   uint8_t* sq2 = smem + kOffQ2;
   uint8_t* sk = smem + kOffK;
   uint8_t* sp = smem + kOffP;
   float* sx = reinterpret_cast<float*>(smem + kOffX);
   float* sl = reinterpret_cast<float*>(smem + kOffL);
+  float* sscale = reinterpret_cast<float*>(smem + kOffScale);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -297,6 +395,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar[kXBar], 32 * kSoftmaxWarps);
     mbar_init(&bar[kLBar], 32 * kSoftmaxWarps);
     for (int i = 0; i < 3; ++i) mbar_init(&bar[kDrain0 + i], 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&bar[kKLanded0 + s], 1);
+      mbar_init(&bar[kVLanded0 + s], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -324,6 +426,9 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   // An idle worker (or bad metadata) runs no role: both CTAs of the pair read
   // the same row and go straight to the common teardown.
+  if constexpr (kFp8) {
+    if (warp >= 8) setmaxnreg_dec<kFp8RegsConv>();
+  }
 
   // Every role walks the same sequence of K-ring entries: per piece with pages,
   // two query-staging entries, then one entry per page.
@@ -427,6 +532,33 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (pending[k] >= 0) warp_arrive_leader(&bar[kKFull0 + pending[k]], rank, lane);
               pending[0] = pending[1] = -1;
             }
+          } else if constexpr (kFp8) {
+            // FP8 codes of this CTA's 32 tokens, one box of 128 bytes x 32 rows x
+            // 9 chunks through a view whose chunks are 64 bytes apart, started at
+            // x = -64: each chunk's codes land in bytes 64..127 of its 128-byte
+            // row slots (bytes 0..63 are zeros, overwritten when the converters
+            // widen the slot); plus the page's 64 scales.  Both count on this
+            // CTA's K-landed barrier; the converters signal the leader's full
+            // barrier.
+            int page = page_next;
+            if (j + 1 < pz.npg) page_next = __ldg(bt + pz.pg0 + j + 1);
+            // the tensor map bounds the codes, but the untiled scale copy has no
+            // bounds: a page id outside the cache is reported and replaced
+            if (page < 0 || page >= p.num_blocks) {
+              report(p.status, MLA_ERR_DEVICE_CHECK);
+              page = 0;
+            }
+            if (use > 0) {
+              ok = wait(&bar[kKEmpty0 + slot], (use - 1) & 1);
+              if (!ok) break;
+            }
+            uint64_t* landed = &bar[kKLanded0 + slot];
+            const int row = page * kPage + 32 * static_cast<int>(rank);
+            mbar_arrive_expect_tx(landed, kChunks * kHalfChunk + kPage * 4);
+            tma_load_3d(sk + slot * kKBytes, &tm_kpart, -64, row, 0, landed);
+            // all 64 tokens' scales: the softmax applies them to both halves of S
+            bulk_load(sscale + slot * kPage, p.kscale + static_cast<int64_t>(page) * kPage,
+                      kPage * 4, landed);
           } else {
             // this page's entry was loaded one page ahead; load the next one
             // before waiting for the slot
@@ -491,6 +623,17 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             cp_async_wait_group<0>();
             fence_proxy_async_smem();
             warp_arrive_leader(&bar[kVFull0 + slot], rank, lane);
+          } else if constexpr (kFp8) {
+            // FP8: the four chunks' codes (one box, as for the K parts) on this
+            // CTA's V-landed barrier; the value converters widen them and signal
+            // the leader's V barrier (the page's scales came with the K part)
+            const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
+            const int page = __ldg(bt + pz.pg0 + j);
+            uint64_t* landed = &bar[kVLanded0 + slot];
+            const int row = page * kPage + src_row;
+            mbar_arrive_expect_tx(landed, kXChunks * kHalfChunk);
+            tma_load_3d(sk + slot * kKBytes + dst_chunk * kHalfChunk, &tm_vx, -64, row, src_chunk,
+                        landed);
           } else {
             const int32_t* bt = p.block_table + static_cast<int64_t>(pz.seq) * p.bt_stride;
             const int page = __ldg(bt + pz.pg0 + j);
@@ -503,6 +646,84 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       if constexpr (kGather) cp_async_wait_group<0>();
+    }
+  } else if (kFp8 && warp >= kKConvWarp0 && warp < kTmaVWarp) {
+    // ------------------------------------------------------------ FP8: K-part converters
+    // Two groups of four warps widen the K parts of even and odd pages, so two
+    // pages are widened at once.  In a group, thread t owns row r = t % 32 of
+    // chunks t / 32, t / 32 + 4, ... (3 or 2 of the 9); the group signals the
+    // leader's full barrier once per page (one arrival per CTA).
+    const int group = (warp - kKConvWarp0) / 4;
+    const int ct = threadIdx.x - (kKConvWarp0 + 4 * group) * 32;
+    const int r = ct & 31, c0 = ct >> 5;
+    const int named = kKConvBarrier0 + group;
+    int entries = 0, pages = 0;
+    uint32_t landed_parity = 0;  // per slot: K parts landed there (mod 2), both groups'
+    for (int pc = 0; pc < npieces; ++pc) {
+      const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+      if (pz.npg == 0) continue;
+      entries += 2;  // the query staging entries go straight to the consumers
+      bool stop = false;
+      for (int j = 0; j < pz.npg; ++j, ++entries) {
+        const int slot = entries % kKSlots;
+        const uint32_t parity = (landed_parity >> slot) & 1;
+        landed_parity ^= 1u << slot;
+        if (((pages + j) % kKConvGroups) != group) continue;
+        if (!convert_wait(&bar[kKLanded0 + slot], parity, abort_flag, wait_ns, named,
+                          kKConvThreads)) {
+          stop = true;
+          break;
+        }
+        uint8_t* row_slot = sk + slot * kKBytes + r * 128;
+        for (int c = c0; c < kChunks; c += 4) widen_row_slot(row_slot + c * kHalfChunk, r);
+        fence_proxy_async_smem();  // the MMAs read the slot through the async proxy
+        named_bar_sync(named, kKConvThreads);
+        if (ct == 0) {
+          if (rank == 0)
+            mbar_arrive(&bar[kKFull0 + slot]);
+          else
+            mbar_arrive_remote(&bar[kKFull0 + slot], 0);
+        }
+      }
+      if (stop) break;
+      pages += pz.npg;
+    }
+  } else if (kFp8 && warp >= kVConvWarp0) {
+    // ------------------------------------------------------------ FP8: value converters
+    // Widen the peer tokens' value chunks: 4 chunks x 32 rows, row slot i
+    // (row i % 32 of chunk i / 32) for i = t and t + 96.
+    const int ct = threadIdx.x - kVConvWarp0 * 32;
+    const int dst_chunk = rank == 0 ? kXChunks : 0;
+    int entries = 0;
+    uint32_t landed_parity = 0;
+    for (int pc = 0; pc < npieces; ++pc) {
+      const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
+      if (pz.npg == 0) continue;
+      entries += 2;
+      bool stop = false;
+      for (int j = 0; j < pz.npg; ++j, ++entries) {
+        const int slot = entries % kKSlots;
+        const uint32_t parity = (landed_parity >> slot) & 1;
+        landed_parity ^= 1u << slot;
+        if (!convert_wait(&bar[kVLanded0 + slot], parity, abort_flag, wait_ns, kVConvBarrier,
+                          kVConvThreads)) {
+          stop = true;
+          break;
+        }
+        for (int i = ct; i < kXChunks * 32; i += kVConvThreads) {
+          const int r = i & 31;
+          widen_row_slot(sk + slot * kKBytes + (dst_chunk + (i >> 5)) * kHalfChunk + r * 128, r);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(kVConvBarrier, kVConvThreads);
+        if (ct == 0) {
+          if (rank == 0)
+            mbar_arrive(&bar[kVFull0 + slot]);
+          else
+            mbar_arrive_remote(&bar[kVFull0 + slot], 0);
+        }
+      }
+      if (stop) break;
     }
   } else if (warp == kQkEvenWarp || warp == kQkOddWarp) {
     // ------------------------------------------------------------ QK^T issuers (leader)
@@ -543,20 +764,46 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint64_t b0 = smem_desc_sw128(k_base + slot * kKBytes, 16, 1024);
           const uint64_t a2 = smem_desc_sw128(q2_base, 16, 1024);
           const uint32_t d = tmem + kTmemS + 32 * b;
+          if constexpr (kFp8) {
+            // the same K-steps, one chunk (four K-steps) per iteration: the
+            // fully unrolled form below needs more registers than the FP8
+            // kernel's issuing warps have (descriptor addresses count 16-byte
+            // units)
+#pragma unroll 1
+            for (int c = 0; c < kChunks; ++c) {
+              const uint64_t bc = b0 + static_cast<uint32_t>((c * kHalfChunk) >> 4);
+              if (c < kQTmemChunks) {
+                const uint32_t ac = tmem + kTmemQ + 32 * c;
 #pragma unroll
-          for (int kk = 0; kk < kQKSteps; ++kk) {
-            // K-step kk: swizzle block kk/4, 32-byte step kk%4 inside it
-            const uint32_t boff = ((kk >> 2) * kHalfChunk + (kk & 3) * 32) >> 4;
-            if (kk < kQTmemKSteps) {
-              umma_bf16_ts_pair(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
-            } else {
-              const int k2 = kk - kQTmemKSteps;
-              const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
-              umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
+                for (int k = 0; k < 4; ++k)
+                  umma_bf16_ts_pair(d, ac + 8 * k, bc + 2 * k, kIdescQK, (c | k) != 0 ? 1u : 0u);
+              } else {
+                const uint64_t ac = a2 + static_cast<uint32_t>(((c - kQTmemChunks) * kChunk) >> 4);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  umma_bf16_ss_pair(d, ac + 2 * k, bc + 2 * k, kIdescQK, 1u);
+              }
+              // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
+              if (4 * c + 3 == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
+              if (4 * c + 3 == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
             }
-            // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
-            if (kk == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
-            if (kk == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kQKSteps; ++kk) {
+              // K-step kk: swizzle block kk/4, 32-byte step kk%4 inside it
+              const uint32_t boff = ((kk >> 2) * kHalfChunk + (kk & 3) * 32) >> 4;
+              if (kk < kQTmemKSteps) {
+                umma_bf16_ts_pair(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK,
+                                  kk > 0 ? 1u : 0u);
+              } else {
+                const int k2 = kk - kQTmemKSteps;
+                const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
+                umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
+              }
+              // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
+              if (kk == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
+              if (kk == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
+            }
           }
           umma_commit_pair(&bar[kSFull0 + b]);
         }
@@ -618,6 +865,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax / epilogue
+    if constexpr (kFp8) setmaxnreg_inc<kFp8RegsSoftmax>();
     const int L = 32 * warp + lane;       // TMEM lane
     const int r = L & 63;                 // row within this CTA's 64
     const int th = L >> 6;                // which half of the 64 tokens / of each dv 256-block
@@ -628,6 +876,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     int entries = 0, pages = 0, pieces_done = 0, qcopies = 0;
     bool ok = true;
     bool q_copied_ahead = false;
+    uint32_t landed_parity = 0;  // FP8: per slot, pages whose codes and scales landed (mod 2)
     for (int pc = 0; pc < npieces && ok; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       const int Lseq = p.seqlens[pz.seq];
@@ -658,11 +907,25 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_before();
           warp_arrive_leader(&bar[kSFree0 + pb], rank, lane);
           const int nv = lim - (pz.pg0 + j) * kPage - 32 * th;
+          // FP8 cache: the MMAs saw the codes; token c's scale multiplies its
+          // score here and its probability below.  The page's scales landed with
+          // this CTA's K part (the barrier's phase is complete: the slot is not
+          // reloaded before PV of this page, which needs this softmax).
+          const float* tsc = sscale;  // FP8: this thread's 32 tokens' scales
+          if constexpr (kFp8) {
+            const int slot = (entries + j) % kKSlots;
+            const uint32_t parity = (landed_parity >> slot) & 1;
+            landed_parity ^= 1u << slot;
+            ok = warp_wait_cluster(&bar[kKLanded0 + slot], parity, abort_flag, wait_ns);
+            if (!ok) break;
+            tsc = sscale + slot * kPage + 32 * th;
+          }
           float x[32];
           float mx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            x[c] = c < nv ? __uint_as_float(s[c]) * p.scale_log2 : -INFINITY;
+            const float sc = kFp8 ? p.scale_log2 * tsc[c] : p.scale_log2;
+            x[c] = c < nv ? __uint_as_float(s[c]) * sc : -INFINITY;
             mx = fmaxf(mx, x[c]);
           }
           // the other half of the row is in lane L ^ 64
@@ -684,7 +947,14 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float p0 = x[c] == -INFINITY ? 0.f : ex2_approx(x[c] - m);
             const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_approx(x[c + 1] - m);
             sum += p0 + p1;
-            pw[c >> 1] = pack_bf16x2(p0, p1);
+            if constexpr (kFp8) {
+              // the value rows are the codes: P carries the scale (a power of
+              // two, so the bf16 rounding of P is unchanged); a masked token
+              // keeps P = 0 whatever its scale holds
+              pw[c >> 1] = pack_bf16x2(p0 == 0.f ? 0.f : p0 * tsc[c], p1 == 0.f ? 0.f : p1 * tsc[c + 1]);
+            } else {
+              pw[c >> 1] = pack_bf16x2(p0, p1);
+            }
           }
           l = l * alpha + sum;
           // O is rescaled only once PV of the previous page is done; the first
@@ -903,30 +1173,44 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
-}  // namespace
 
-cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
-                               const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
-                               const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
-                               cudaStream_t stream) {
-  static std::atomic<bool> configured[64];  // per device: attribute set (both variants)
+// Shared memory attribute of the three variants (once per device), and the
+// register count the FP8 variant's setmaxnreg split relies on: with fewer
+// registers at launch than its warpgroups ask for in all, the softmax
+// warpgroup's increase could never be granted.
+cudaError_t configure_pair_kernels() {
+  static std::atomic<bool> configured[64];  // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(mla_decode_pair_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (configured[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const void* kernels[3] = {reinterpret_cast<const void*>(mla_decode_pair_kernel<false, false>),
+                            reinterpret_cast<const void*>(mla_decode_pair_kernel<true, false>),
+                            reinterpret_cast<const void*>(mla_decode_pair_kernel<false, true>)};
+  for (const void* k : kernels) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(mla_decode_pair_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev].store(true, std::memory_order_release);
   }
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, kernels[2]);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kFp8LaunchRegs) return cudaErrorInvalidConfiguration;
+  configured[dev].store(true, std::memory_order_release);
+  return cudaSuccess;
+}
+
+template <bool kGather, bool kFp8>
+cudaError_t launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
+                        const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
+                        const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
+                        cudaStream_t stream) {
+  cudaError_t e = configure_pair_kernels();
+  if (e != cudaSuccess) return e;
   const int blocks128 = (p.rows + 127) / 128;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * num_workers, blocks128, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(PairRoles<kFp8>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -938,14 +1222,28 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (p.gather_rows != nullptr)
-    e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel<true>, tm_q, tm_kpart, tm_vx, tm_po,
-                           tm_out, p);
-  else
-    e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel<false>, tm_q, tm_kpart, tm_vx, tm_po,
-                           tm_out, p);
+  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel<kGather, kFp8>, tm_q, tm_kpart, tm_vx,
+                         tm_po, tm_out, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kpart,
+                               const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
+                               const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
+                               cudaStream_t stream) {
+  if (p.gather_rows != nullptr)
+    return launch_pair<true, false>(tm_q, tm_kpart, tm_vx, tm_po, tm_out, p, num_workers, stream);
+  return launch_pair<false, false>(tm_q, tm_kpart, tm_vx, tm_po, tm_out, p, num_workers, stream);
+}
+
+cudaError_t launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_k8,
+                                   const CUtensorMap& tm_v8, const CUtensorMap& tm_po,
+                                   const CUtensorMap& tm_out, const DecodeParams& p,
+                                   int num_workers, cudaStream_t stream) {
+  return launch_pair<false, true>(tm_q, tm_k8, tm_v8, tm_po, tm_out, p, num_workers, stream);
 }
 
 // Pairs (clusters of 2) of this kernel that fit on the device at once.
@@ -960,12 +1258,11 @@ cudaError_t pair_kernel_max_clusters(int* clusters) {
     *clusters = known;
     return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(mla_decode_pair_kernel<false>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = configure_pair_kernels();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(PairRoles<false>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -975,7 +1272,7 @@ cudaError_t pair_kernel_max_clusters(int* clusters) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel<false>, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, mla_decode_pair_kernel<false, false>, &cfg);
   if (e != cudaSuccess) return e;
   if (n < 1) n = 1;
   cached[dev].store(n, std::memory_order_release);

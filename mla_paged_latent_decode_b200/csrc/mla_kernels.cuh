@@ -114,9 +114,9 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_workers, 
 cudaError_t launch_decode(const CUtensorMap& tm_q, const CUtensorMap& tm_page,
                           const DecodeParams& p, int num_workers, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
-// FP8 (E4M3) cache, any number of query rows (one CTA per worker and 64-row
-// block): tm_page8 views the codes as [rows, 576] bytes in boxes of 128 bytes x
-// 64 rows; scales via p.kscale.
+// FP8 (E4M3) cache on single CTAs (one CTA per worker and 64-row block):
+// tm_page8 views the codes as [rows, 576] bytes in boxes of 128 bytes x 64
+// rows; scales via p.kscale.
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_page8,
                               const DecodeParams& p, int num_workers, cudaStream_t stream);
 // Pair kernel (more than 64 query rows per sequence): clusters of 2 CTAs.
@@ -126,6 +126,13 @@ cudaError_t launch_decode_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kp
                                const CUtensorMap& tm_vx, const CUtensorMap& tm_po,
                                const CUtensorMap& tm_out, const DecodeParams& p, int num_workers,
                                cudaStream_t stream);
+// The pair kernel over an FP8 (E4M3) cache: tm_k8 and tm_v8 view the codes as
+// {128 bytes, rows, 9 chunks} with a 64-byte chunk stride, in boxes of 32 rows
+// x 9 and x 4 chunks (started at x = -64); scales via p.kscale.
+cudaError_t launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_k8,
+                                   const CUtensorMap& tm_v8, const CUtensorMap& tm_po,
+                                   const CUtensorMap& tm_out, const DecodeParams& p,
+                                   int num_workers, cudaStream_t stream);
 cudaError_t pair_kernel_max_clusters(int* clusters);
 // Merge of decode results over disjoint parts of the cache (mla_merge.cu):
 // outs [parts, nrows, 512] bf16, lses [parts, b, h_q, s_q] fp32.
