@@ -569,9 +569,9 @@ def run_cuda(args, rank, local, world):
     # end to end through the public API, as a serving loop runs it: every step
     # copies its inputs in from pinned host memory and its outputs back, all
     # inside the timed region.  Three streams (copies in, compute, copies out)
-    # and two sets of step buffers let step k + 1's inputs travel while step k
-    # computes and step k - 1's outputs travel back; the latent cache (larger
-    # than L2) stays resident in HBM, as in serving.
+    # and several sets of step buffers (--e2e-sets) let step k + 1's inputs
+    # travel while step k computes and step k - 1's outputs travel back; the
+    # latent cache (larger than L2) stays resident in HBM, as in serving.
     e2e = None
     if not args.no_e2e:
         n_e2e = max(3, min(args.steps, 200))
@@ -580,7 +580,8 @@ def run_cuda(args, rank, local, world):
         hsl = inp.cache_seqlens.pin_memory()
         hidx = sparse_idx.pin_memory() if sparse_idx is not None else None
         sets = []
-        for _ in range(2):
+        n_sets = max(2, args.e2e_sets)
+        for _ in range(n_sets):
             sets.append(dict(
                 q=torch.empty_like(q), bt=torch.empty_like(bt), sl=torch.empty_like(sl),
                 idx=torch.empty_like(idx_d) if sparse_idx is not None else None,
@@ -598,10 +599,10 @@ def run_cuda(args, rank, local, world):
                 st.wait_stream(stream)
             t0.record(s_in)
             for k in range(n):
-                b = sets[k % 2]
+                b = sets[k % n_sets]
                 with torch.cuda.stream(s_in):
-                    if k >= 2:  # step k - 2 has finished reading this set's inputs
-                        s_in.wait_event(ev_cmp[k - 2])
+                    if k >= n_sets:  # the set's previous step has finished reading its inputs
+                        s_in.wait_event(ev_cmp[k - n_sets])
                     b["q"].copy_(hq, non_blocking=True)
                     b["bt"].copy_(hbt, non_blocking=True)
                     b["sl"].copy_(hsl, non_blocking=True)
@@ -610,8 +611,8 @@ def run_cuda(args, rank, local, world):
                     ev_in[k].record(s_in)
                 with torch.cuda.stream(s_cmp):
                     s_cmp.wait_event(ev_in[k])
-                    if k >= 2:  # step k - 2's outputs in this set have been copied out
-                        s_cmp.wait_event(ev_out[k - 2])
+                    if k >= n_sets:  # the set's previous outputs have been copied out
+                        s_cmp.wait_event(ev_out[k - n_sets])
                     if hidx is not None:
                         binding.mla_decode_sparse(b["q"], kc, b["bt"], b["sl"], b["idx"], inp.scale,
                                                   inp.causal, out=b["out"], lse=b["lse"],
@@ -644,20 +645,46 @@ def run_cuda(args, rank, local, world):
         e2e_total = reduce_max(run_e2e(n_e2e), world, dev)
         e2e_bytes = reduce_sum(float(nbytes * n_e2e), world, dev)
         # the last step's outputs arrived intact
-        if not torch.equal(sets[(n_e2e - 1) % 2]["hout"], out.cpu()):
+        if not torch.equal(sets[(n_e2e - 1) % n_sets]["hout"], out.cpu()):
             raise RuntimeError("end-to-end output differs from the device-timed output")
         h2d = hq.numel() * hq.element_size() + hbt.numel() * 4 + hsl.numel() * 4
         if sparse_idx is not None:
             h2d += sparse_idx.numel() * 4
         d2h = out.numel() * out.element_size() + lse.numel() * 4
+        # the host link on its own: the step's input copy and output copy, each
+        # alone and both at once (one per direction), best of five
+        def link_us(copy_in, copy_out):
+            best = float("inf")
+            for _ in range(5):
+                for st in (s_in, s_out):
+                    st.wait_stream(stream)
+                a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s_in)
+                s_out.wait_event(a)
+                if copy_in:
+                    with torch.cuda.stream(s_in):
+                        sets[0]["q"].copy_(hq, non_blocking=True)
+                if copy_out:
+                    with torch.cuda.stream(s_out):
+                        sets[0]["hout"].copy_(sets[0]["out"], non_blocking=True)
+                s_in.wait_stream(s_out)
+                z.record(s_in)
+                torch.cuda.synchronize(dev)
+                best = min(best, a.elapsed_time(z) * 1e3)
+            return best
+        h2d_us, d2h_us, both_us = link_us(True, False), link_us(False, True), link_us(True, True)
         e2e = {"value": e2e_bytes / e2e_total / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "us_per_step": e2e_total / n_e2e * 1e6,
+               "us_per_step": e2e_total / n_e2e * 1e6, "buffer_sets": n_sets,
+               "link": {"q_in_us": h2d_us, "out_back_us": d2h_us, "both_us": both_us,
+                        "h2d_gb_s": hq.numel() * hq.element_size() / h2d_us / 1e3,
+                        "d2h_gb_s": out.numel() * out.element_size() / d2h_us / 1e3},
                "note": "through the public API: q, block_table and cache_seqlens copied in from "
                        "pinned host memory and out and lse copied back every step; copies in, "
-                       "compute and copies out on three streams with two buffer sets, so "
+                       f"compute and copies out on three streams with {n_sets} buffer sets, so "
                        "consecutive steps overlap; the latent cache stays resident in HBM as "
-                       "in serving"}
+                       "in serving; link: the q copy in and the out copy back timed alone and "
+                       "together"}
 
     append = None if args.no_append else measure_append(inp, dev, stream, flush_l2, fp8=fp8)
 
@@ -840,6 +867,9 @@ def main():
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
                     help="latent cache format (fp8: E4M3 codes + per-token scale)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
+    ap.add_argument("--e2e-sets", type=int, default=4,
+                    help="step buffer sets of the end-to-end loop (copies of consecutive steps "
+                         "overlap across them)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
     ap.add_argument("--sparse-topk", type=int, default=0,
                     help="time the sparse decode with this many selected tokens per query "
