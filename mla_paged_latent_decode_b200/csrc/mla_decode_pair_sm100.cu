@@ -310,6 +310,33 @@ __device__ __forceinline__ void widen_row_slot(uint8_t* slot, int r) {
   }
 }
 
+// The MMA-issuing roles run either on a whole warp (kWarp: every lane runs the
+// loop, one elected lane issues each MMA and commit) or on lane 0 alone.
+template <bool kWarp>
+__device__ __forceinline__ bool issuer_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            uint64_t limit_ns) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort, limit_ns);
+  if constexpr (kWarp) return __all_sync(0xffffffffu, ok);
+  return ok;
+}
+template <bool kWarp>
+__device__ __forceinline__ void issue_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+  if constexpr (kWarp) umma_bf16_ts_pair_warp(d, a, b, idesc, acc);
+  else umma_bf16_ts_pair(d, a, b, idesc, acc);
+}
+template <bool kWarp>
+__device__ __forceinline__ void issue_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+  if constexpr (kWarp) umma_bf16_ss_pair_warp(d, a, b, idesc, acc);
+  else umma_bf16_ss_pair(d, a, b, idesc, acc);
+}
+template <bool kWarp>
+__device__ __forceinline__ void issue_commit(uint64_t* bar) {
+  if constexpr (kWarp) umma_commit_pair_warp(bar);
+  else umma_commit_pair(bar);
+}
+
 // Gathered rows: copy 32 cached rows (this lane holds the row index of row
 // `lane`; -1 = a zero row) into a slot, chunks src_chunk .. src_chunk +
 // nchunks - 1 of each row to chunks dst_chunk .. of the slot, in the
@@ -350,6 +377,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   // pages), or one arrival per CTA (gathered rows, copied by the threads; FP8
   // codes, widened by the converter warps)
   constexpr uint32_t kFullArrivals = (kGather || kFp8) ? 2 : 1;
+  constexpr bool kWarpIssue = !kFp8;  // MMAs issued by whole warps (see the QK^T issuers)
   (void)kThreads;
   uint8_t* sq2 = smem + kOffQ2;
   uint8_t* sk = smem + kOffK;
@@ -727,9 +755,12 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kQkEvenWarp || warp == kQkOddWarp) {
     // ------------------------------------------------------------ QK^T issuers (leader)
-    // One thread issues a tcgen05.mma at most every ~45 cycles; even and odd
+    // With a bf16 cache each warp issues as a whole (every lane runs the loop,
+    // one elected lane issues each MMA and commit): about one MMA per 27 cycles
+    // against 60 for a single thread.  The FP8 variant issues from lane 0 (with
+    // its fewer registers the whole-warp form measured slower).  Even and odd
     // pages (one S buffer each) come from two warps so the tensor core stays fed.
-    if (rank == 0 && lane == 0) {
+    if (rank == 0 && (kWarpIssue || lane == 0)) {
       const int parity = warp == kQkEvenWarp ? 0 : 1;
       int entries = 0, pages = 0, qloads = 0;
       bool ok = true;
@@ -739,25 +770,25 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (pz.npg == 0) continue;
         const int stage_a = entries % kKSlots, stage_b = (entries + 1) % kKSlots;
         entries += 2;
-        ok = mbar_wait_cluster(&bar[kQFull], qloads & 1, abort_flag, wait_ns) &&
-             mbar_wait_cluster(&bar[kQReady], qloads & 1, abort_flag, wait_ns);
+        ok = issuer_wait<kWarpIssue>(&bar[kQFull], qloads & 1, abort_flag, wait_ns) &&
+             issuer_wait<kWarpIssue>(&bar[kQReady], qloads & 1, abort_flag, wait_ns);
         ++qloads;
         if (!ok) break;
         tc_fence_after();
         if (parity == 0) {  // both CTAs hold Q in tensor memory: the staging slots are free
-          umma_commit_pair(&bar[kKEmpty0 + stage_a]);
-          umma_commit_pair(&bar[kKEmpty0 + stage_b]);
+          issue_commit<kWarpIssue>(&bar[kKEmpty0 + stage_a]);
+          issue_commit<kWarpIssue>(&bar[kKEmpty0 + stage_b]);
         }
         for (int j = 0; j < pz.npg && ok; ++j) {
           const int g = pages + j, b = g & 1, entry = entries + j;
           if (b != parity) continue;
           if (g >= 2) {  // both CTAs' softmax have read S of page g - 2 from buffer b
-            ok = mbar_wait_cluster(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag,
+            ok = issuer_wait<kWarpIssue>(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag,
                                    wait_ns);
             if (!ok) break;
           }
           const int slot = entry % kKSlots;
-          ok = mbar_wait_cluster(&bar[kKFull0 + slot], (entry / kKSlots) & 1, abort_flag,
+          ok = issuer_wait<kWarpIssue>(&bar[kKFull0 + slot], (entry / kKSlots) & 1, abort_flag,
                                  wait_ns);
           if (!ok) break;
           tc_fence_after();
@@ -776,16 +807,16 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const uint32_t ac = tmem + kTmemQ + 32 * c;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                  umma_bf16_ts_pair(d, ac + 8 * k, bc + 2 * k, kIdescQK, (c | k) != 0 ? 1u : 0u);
+                  issue_ts<kWarpIssue>(d, ac + 8 * k, bc + 2 * k, kIdescQK, (c | k) != 0 ? 1u : 0u);
               } else {
                 const uint64_t ac = a2 + static_cast<uint32_t>(((c - kQTmemChunks) * kChunk) >> 4);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                  umma_bf16_ss_pair(d, ac + 2 * k, bc + 2 * k, kIdescQK, 1u);
+                  issue_ss<kWarpIssue>(d, ac + 2 * k, bc + 2 * k, kIdescQK, 1u);
               }
               // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
-              if (4 * c + 3 == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
-              if (4 * c + 3 == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
+              if (4 * c + 3 == kXDoneStep0) issue_commit<kWarpIssue>(&bar[kXFree0 + 2 * slot]);
+              if (4 * c + 3 == kXDoneStep1) issue_commit<kWarpIssue>(&bar[kXFree0 + 2 * slot + 1]);
             }
           } else {
 #pragma unroll
@@ -793,29 +824,29 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
               // K-step kk: swizzle block kk/4, 32-byte step kk%4 inside it
               const uint32_t boff = ((kk >> 2) * kHalfChunk + (kk & 3) * 32) >> 4;
               if (kk < kQTmemKSteps) {
-                umma_bf16_ts_pair(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK,
+                issue_ts<kWarpIssue>(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK,
                                   kk > 0 ? 1u : 0u);
               } else {
                 const int k2 = kk - kQTmemKSteps;
                 const uint32_t aoff = ((k2 >> 2) * kChunk + (k2 & 3) * 32) >> 4;
-                umma_bf16_ss_pair(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
+                issue_ss<kWarpIssue>(d, a2 + aoff, b0 + boff, kIdescQK, 1u);
               }
               // chunks 0..3 / 4..7 of the slot read: the peer-token values may land there
-              if (kk == kXDoneStep0) umma_commit_pair(&bar[kXFree0 + 2 * slot]);
-              if (kk == kXDoneStep1) umma_commit_pair(&bar[kXFree0 + 2 * slot + 1]);
+              if (kk == kXDoneStep0) issue_commit<kWarpIssue>(&bar[kXFree0 + 2 * slot]);
+              if (kk == kXDoneStep1) issue_commit<kWarpIssue>(&bar[kXFree0 + 2 * slot + 1]);
             }
           }
-          umma_commit_pair(&bar[kSFull0 + b]);
+          issue_commit<kWarpIssue>(&bar[kSFull0 + b]);
         }
         if (!ok) break;
-        umma_commit_pair(&bar[kQEmpty]);  // this warp's reads of Q for the piece are done
+        issue_commit<kWarpIssue>(&bar[kQEmpty]);  // this warp's reads of Q for the piece are done
         entries += pz.npg;
         pages += pz.npg;
       }
     }
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------ PV issuer (leader)
-    if (rank == 0 && lane == 0) {
+    if (rank == 0 && (kWarpIssue || lane == 0)) {  // as for QK^T
       int pages = 0, entries = 0;
       uint32_t vbits = 0;  // parity of the next phase of each slot's V barrier
       bool ok = true;
@@ -826,14 +857,15 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         entries += 2;  // the piece's query staging entries
         for (int j = 0; j < pz.npg; ++j, ++entries) {
           const int g = pages + j, slot = entries % kKSlots, pb = g & 1;
-          ok = mbar_wait_cluster(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, wait_ns);
+          ok = issuer_wait<kWarpIssue>(&bar[kPFull0 + pb], (g >> 1) & 1, abort_flag, wait_ns);
           if (!ok) break;
           // test hook: a wait that nothing ends, with copies and MMAs in flight
           if (g == 0 && p.stall_flag != nullptr) {
             ok = flag_wait(p.stall_flag, abort_flag, wait_ns);
+            if constexpr (kWarpIssue) ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
           }
-          ok = mbar_wait_cluster(&bar[kVFull0 + slot], (vbits >> slot) & 1u, abort_flag,
+          ok = issuer_wait<kWarpIssue>(&bar[kVFull0 + slot], (vbits >> slot) & 1u, abort_flag,
                                  wait_ns);
           if (!ok) break;
           vbits ^= 1u << slot;
@@ -850,16 +882,16 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
               // (LBO = one 32-row chunk, SBO = 8 rows)
               const uint32_t vaddr = st + ((kk >> 1) * kXChunks + 2 * h) * kHalfChunk +
                                      (kk & 1) * 2048;
-              umma_bf16_ss_pair(tmem + kTmemO + 128 * h, smem_desc_sw128(pt + kk * 32, 16, 1024),
+              issue_ss<kWarpIssue>(tmem + kTmemO + 128 * h, smem_desc_sw128(pt + kk * 32, 16, 1024),
                                 smem_desc_sw128(vaddr, kHalfChunk, 1024), kIdescPV,
                                 (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          umma_commit_pair(&bar[kKEmpty0 + slot]);
-          umma_commit_pair(&bar[kPvDone0 + pb]);
+          issue_commit<kWarpIssue>(&bar[kKEmpty0 + slot]);
+          issue_commit<kWarpIssue>(&bar[kPvDone0 + pb]);
         }
         if (!ok) break;
-        umma_commit_pair(&bar[kOFull]);
+        issue_commit<kWarpIssue>(&bar[kOFull]);
         pages += pz.npg;
       }
     }
@@ -1156,10 +1188,17 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   // within microseconds; a grace period covers them).  Both must be done before
   // the shared and tensor memory they write is released at the exit.
   if (*abort_flag) {
-    if (rank == 0 && lane == 0 && warp >= kQkEvenWarp && warp <= kQkOddWarp) {
+    if (rank == 0 && warp >= kQkEvenWarp && warp <= kQkOddWarp) {
+      // the lane that issued the MMAs commits (the elected one of a whole warp)
       uint64_t* db = &bar[kDrain0 + (warp - kQkEvenWarp)];
-      umma_commit_leader(db);
-      mbar_wait_drain(db, 0, kWaitLimitNs);
+      __syncwarp();
+      if constexpr (kWarpIssue) {
+        umma_commit_leader_warp(db);
+        mbar_wait_drain(db, 0, kWaitLimitNs);
+      } else if (lane == 0) {
+        umma_commit_leader(db);
+        mbar_wait_drain(db, 0, kWaitLimitNs);
+      }
     }
     if (threadIdx.x == 0) abort_grace();
   }

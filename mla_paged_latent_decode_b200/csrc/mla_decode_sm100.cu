@@ -114,6 +114,21 @@ struct Piece {
   int seq, pg0, npg, split_idx;
 };
 
+// The MMA-issuing roles run either on a whole warp (kWarp: every lane runs the
+// loop, one elected lane issues each MMA and commit) or on lane 0 alone.
+template <bool kWarp>
+__device__ __forceinline__ bool issuer_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  if constexpr (kWarp) return __all_sync(0xffffffffu, ok);
+  return ok;
+}
+template <bool kWarp>
+__device__ __forceinline__ void issue_commit(uint64_t* bar) {
+  if constexpr (kWarp) umma_commit_warp(bar);
+  else umma_commit(bar);
+}
+
 // Piece `pc` of a worker: its sequence, first page, page count and split index.
 // The page count never exceeds the block-table row (bt_stride entries).
 __device__ __forceinline__ Piece piece_of(const int32_t* md, int pc, const int32_t* seqlens,
@@ -155,6 +170,9 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   constexpr int kSFull0 = C::kSFull0, kSFull1 = C::kSFull1, kSFree0 = C::kSFree0;
   constexpr int kSFree1 = C::kSFree1, kPFull = C::kPFull, kPvDone = C::kPvDone;
   constexpr int kOFull = C::kOFull;
+  // MMAs issued by whole warps with a bf16 cache; from lane 0 in the FP8
+  // variant, whose issuing warps run with 56 registers
+  constexpr bool kWarpIssue = !kFp8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -471,12 +489,14 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kMmaWarp || warp == kQkOddWarp) {
     // ------------------------------------------------------------ QK^T issuers
-    // A single thread issues a tcgen05.mma only every ~45 cycles, longer than an
+    // A single thread issues a tcgen05.mma only every ~60 cycles, longer than an
     // M=64 N=64 MMA takes.  So QK^T of even pages (S buffer 0), QK^T of odd
     // pages (S buffer 1) and PV come from three warps, and the tensor core runs
-    // their MMAs back to back.  QK^T runs up to two pages ahead of the softmax.
+    // their MMAs back to back; with a bf16 cache each warp issues as a whole
+    // (every lane runs the loop, an elected lane issues), which is faster still.
+    // QK^T runs up to two pages ahead of the softmax.
     const int parity = warp == kMmaWarp ? 0 : 1;
-    if (lane == 0) {
+    if (kWarpIssue || lane == 0) {
       int entries = 0, pages = 0, qloads = 0;
       bool ok = true;
       const uint32_t kv_base = smem_addr(skv);
@@ -486,20 +506,21 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int q_entry = entries;   // copied into TMEM by the softmax warps
         const int first = entries + 1;
         entries += 1 + pz.npg;
-        ok = mbar_wait(&bar[kQFull], qloads & 1, abort_flag, wait_ns);
+        ok = issuer_wait<kWarpIssue>(&bar[kQFull], qloads & 1, abort_flag, wait_ns);
         ++qloads;
         if (!ok) break;
-        if (parity == 0) mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // query stage free
+        if (parity == 0 && lane == 0) mbar_arrive(&bar[kEmpty0 + q_entry % kStages]);  // query stage free
         tc_fence_after();
         for (int j = 0; j < pz.npg && ok; ++j) {
           const int g = pages + j, b = g & 1;
           if (b != parity) continue;
           if (g >= 2) {  // the softmax has read S of page g - 2 from buffer b
-            ok = mbar_wait(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag, wait_ns);
+            ok = issuer_wait<kWarpIssue>(&bar[kSFree0 + b], ((g >> 1) - 1) & 1, abort_flag, wait_ns);
             if (!ok) break;
           }
           const int entry = first + j, stage = entry % kStages;
-          ok = mbar_wait(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag, wait_ns);
+          ok = issuer_wait<kWarpIssue>(&bar[kFull0 + stage], (entry / kStages) & 1, abort_flag,
+                                       wait_ns);
           if (!ok) break;
           tc_fence_after();
           const uint64_t b0 = smem_desc_sw128(kv_base + stage * kTileBytes, 16, 1024);
@@ -508,16 +529,19 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int kk = 0; kk < kDqk / 16; ++kk) {
             // K-step kk: swizzle block kk/4, 32-byte step (kk%4) inside it
             const uint32_t boff = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-            umma_bf16_ts(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
+            if constexpr (kWarpIssue)
+              umma_bf16_ts_warp(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
+            else
+              umma_bf16_ts(d, tmem + kTmemQ + 8 * kk, b0 + boff, kIdescQK, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&bar[kSFull0 + b]);
+          issue_commit<kWarpIssue>(&bar[kSFull0 + b]);
         }
         pages += pz.npg;
       }
     }
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------ PV issuer
-    if (lane == 0) {
+    if (kWarpIssue || lane == 0) {  // as for QK^T
       int entries = 0, pages = 0;
       bool ok = true;
       const uint32_t kv_base = smem_addr(skv), p_base = smem_addr(sp);
@@ -530,11 +554,12 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int g = pages + j;
           // P of page g is in shared memory (and QK^T of page g, which read the
           // same stage, has completed: the softmax saw its S)
-          ok = mbar_wait(&bar[kPFull], g & 1, abort_flag, wait_ns);
+          ok = issuer_wait<kWarpIssue>(&bar[kPFull], g & 1, abort_flag, wait_ns);
           if (!ok) break;
           // test hook: a wait that nothing ends, with copies and MMAs in flight
           if (g == 0 && p.stall_flag != nullptr) {
             ok = flag_wait(p.stall_flag, abort_flag, wait_ns);
+            if constexpr (kWarpIssue) ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
           }
           tc_fence_after();
@@ -545,19 +570,24 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int half = 0; half < 2; ++half) {
 #pragma unroll
             for (int kk = 0; kk < kPage / 16; ++kk) {
-              umma_bf16_ss(tmem + kTmemO + half * 256, smem_desc_sw128(p_base + kk * 32, 16, 1024),
-                           smem_desc_sw128(tile + half * 4 * kChunkBytes + kk * 2048,
-                                           kChunkBytes, 1024),
-                           kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+              const uint64_t pa = smem_desc_sw128(p_base + kk * 32, 16, 1024);
+              const uint64_t vb =
+                  smem_desc_sw128(tile + half * 4 * kChunkBytes + kk * 2048, kChunkBytes, 1024);
+              if constexpr (kWarpIssue)
+                umma_bf16_ss_warp(tmem + kTmemO + half * 256, pa, vb, kIdescPV,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+              else
+                umma_bf16_ss(tmem + kTmemO + half * 256, pa, vb, kIdescPV,
+                             (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          umma_commit(&bar[kEmpty0 + stage]);
-          umma_commit(&bar[kPvDone]);
+          issue_commit<kWarpIssue>(&bar[kEmpty0 + stage]);
+          issue_commit<kWarpIssue>(&bar[kPvDone]);
         }
         if (!ok) break;
         // every MMA of the piece is complete once this fires: the last PV
         // follows (through the softmax) the last QK^T
-        umma_commit(&bar[kOFull]);
+        issue_commit<kWarpIssue>(&bar[kOFull]);
         pages += pz.npg;
       }
     }
@@ -775,9 +805,11 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   // thread waits for its own through a commit before tensor and shared memory
   // are released (the TMA producer has already let its copies land).
   if (*abort_flag) {
-    if (lane == 0 && (warp == kMmaWarp || warp == kPvWarp || warp == kQkOddWarp)) {
+    if ((kWarpIssue || lane == 0) && (warp == kMmaWarp || warp == kPvWarp || warp == kQkOddWarp)) {
+      // the lane that issued the MMAs commits (the elected one of a whole warp)
       uint64_t* db = &bar[C::kDrain0 + (warp - kMmaWarp)];
-      umma_commit(db);
+      if constexpr (kWarpIssue) __syncwarp();
+      issue_commit<kWarpIssue>(db);
       mbar_wait_drain(db, 0, kWaitLimitNs);
     }
     if (threadIdx.x == 0) abort_grace();
