@@ -183,20 +183,14 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
-  // Launched as a programmatic dependent of the scheduler kernel: its CTAs may
-  // start while the scheduler runs, and read the metadata only after this wait.
-  grid_dependency_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int worker = blockIdx.x, rb = blockIdx.y;
   const uint64_t wait_ns = p.wait_ns;  // limit of every bounded wait (normally kWaitLimitNs)
-  const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
-  const int npieces = md[5];
-  if (npieces == 0) return;  // idle worker: uniform exit before any barrier or TMEM use
-  if (md[0] < 0 || npieces < 0 || md[0] + npieces > p.batch) {  // metadata not from this batch
-    if (threadIdx.x == 0) report(p.status, MLA_ERR_DEVICE_CHECK);
-    return;
-  }
 
+  // Set-up first: the kernel is launched as a programmatic dependent of the
+  // scheduler kernel, so its CTAs may start while the scheduler runs; barriers
+  // and tensor memory are made ready meanwhile, and the metadata is read only
+  // after the dependency wait below.
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar[kFull0 + s], 1);
@@ -225,6 +219,16 @@ mla_decode_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  grid_dependency_wait();  // the scheduler's metadata is complete and visible
+  const int32_t* md = p.tile_md + static_cast<int64_t>(worker) * kMdStride;
+  int npieces = md[5];
+  if (npieces != 0 && (md[0] < 0 || npieces < 0 || md[0] + npieces > p.batch)) {
+    if (threadIdx.x == 0) report(p.status, MLA_ERR_DEVICE_CHECK);  // metadata not from this batch
+    npieces = 0;
+  }
+  // An idle worker (or bad metadata) runs no role and goes straight to the
+  // common teardown.
   // FP8 cache: 512 threads launched with 128 registers each; the softmax
   // warpgroup raises its budget to 232, the single-thread roles (warps 4-7)
   // lower theirs to 56 and the two converter warpgroups to 96: 61440 of the
