@@ -590,6 +590,8 @@ def run_cuda(args, rank, local, world):
                 hlse=torch.empty(lse.shape, dtype=lse.dtype).pin_memory()))
         s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
 
+        host_enqueue_s = [0.0]
+
         def run_e2e(n):
             ev_in = [torch.cuda.Event() for _ in range(n)]
             ev_cmp = [torch.cuda.Event() for _ in range(n)]
@@ -598,6 +600,7 @@ def run_cuda(args, rank, local, world):
             for st in (s_in, s_cmp, s_out):
                 st.wait_stream(stream)
             t0.record(s_in)
+            h0 = time.perf_counter()
             for k in range(n):
                 b = sets[k % n_sets]
                 with torch.cuda.stream(s_in):
@@ -633,6 +636,7 @@ def run_cuda(args, rank, local, world):
                     b["hout"].copy_(b["out"], non_blocking=True)
                     b["hlse"].copy_(b["lse"], non_blocking=True)
                     ev_out[k].record(s_out)
+            host_enqueue_s[0] = time.perf_counter() - h0  # the host's work for the n steps
             s_out.wait_stream(s_in)
             s_out.wait_stream(s_cmp)
             t1.record(s_out)
@@ -676,6 +680,7 @@ def run_cuda(args, rank, local, world):
         e2e = {"value": e2e_bytes / e2e_total / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "us_per_step": e2e_total / n_e2e * 1e6, "buffer_sets": n_sets,
+               "host_enqueue_us_per_step": host_enqueue_s[0] / n_e2e * 1e6,
                "link": {"q_in_us": h2d_us, "out_back_us": d2h_us, "both_us": both_us,
                         "h2d_gb_s": hq.numel() * hq.element_size() / h2d_us / 1e3,
                         "d2h_gb_s": out.numel() * out.element_size() / d2h_us / 1e3},
