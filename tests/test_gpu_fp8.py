@@ -104,9 +104,10 @@ def test_fp8_full_size_128_heads(cuda_device, name):
     assert_close_lse(lse, ref_lse, "fp8 lse")
 
 
-@pytest.mark.parametrize("num_workers", [1, 3, 17, 600])
-def test_fp8_decode_forced_splits(cuda_device, num_workers):
-    w = synth.custom_workload(3, 2, 16, [700, 5, 1100], causal=True)
+@pytest.mark.parametrize("num_workers,h_q", [(1, 16), (3, 16), (17, 16), (600, 16), (2, 128),
+                                             (9, 128), (74, 128)])
+def test_fp8_decode_forced_splits(cuda_device, num_workers, h_q):
+    w = synth.custom_workload(3, 2, h_q, [700, 5, 1100], causal=True)
     inp = synth.make_inputs(w, seed=31)
     codes, scales = encode_cache(inp.kcache)
     out, lse, md, ns = run_fp8(inp, codes, scales, cuda_device, num_workers)
@@ -116,10 +117,13 @@ def test_fp8_decode_forced_splits(cuda_device, num_workers):
     assert_close_lse(lse, ref_lse, "fp8 lse")
 
 
-def test_fp8_decode_ignores_stale_tail_rows(cuda_device):
+@pytest.mark.parametrize("h_q", [16, 128])
+def test_fp8_decode_ignores_stale_tail_rows(cuda_device, h_q):
     # rows past each sequence's end hold NaN codes and infinite scales: the
-    # kernel must never let them reach an output
-    w = synth.custom_workload(3, 1, 16, [37, 64, 100])
+    # kernel must never let them reach an output (16 heads: single CTAs, which
+    # zero such rows; 128 heads: CTA pairs, which mask their scores and give
+    # them zero probability whatever their scale holds)
+    w = synth.custom_workload(3, 1, h_q, [37, 64, 100])
     inp = synth.make_inputs(w, seed=32)
     codes, scales = encode_cache(inp.kcache)
     ref_out, ref_lse = oracle.decode(inp.q, dequantized(codes, scales), inp.block_table,
