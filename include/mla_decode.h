@@ -272,15 +272,13 @@ int mla_append_latent_fp8(const void* rows, int s_new, void* kcache, float* ksca
  *
  * kcache:  device uint8 [num_blocks, 64, 576] E4M3 codes, 16-byte aligned.
  * kscale:  device fp32 [num_blocks, 64] per-token scales, 16-byte aligned.
- * Rows of a sequence's last page past its length are never read as data
- * (zeroed, or masked with zero probability), so their codes and scales may
- * hold anything.  Widening is exact for scales 2^k with -124 <= k <= 67 (what
+ * Rows of a sequence's last page past its length are never read as data (the
+ * kernels zero them), so their codes and scales may hold anything.  Widening is exact for scales 2^k with -124 <= k <= 67 (what
  * the quantising append writes for rows whose largest magnitude lies in about
  * [1e-35, 6.6e22]).  Any s_q * h_q up to 65536 (MLA_ERR_UNSUPPORTED above):
- * up to 64 query rows per sequence on single CTAs (codes widened to code *
- * scale), more on CTA pairs like mla_decode_kvcache (codes widened to their
- * values, each token's scale applied to its score and, exactly, to its
- * probability).  Metadata from mla_get_metadata as for mla_decode_kvcache.
+ * up to 64 query rows per sequence on single CTAs, more on CTA pairs like
+ * mla_decode_kvcache; both widen the codes to code * scale.  Metadata from
+ * mla_get_metadata as for mla_decode_kvcache.
  * All other arguments, the workspace, errors and launches are as for
  * mla_decode_kvcache.
  */

@@ -65,11 +65,10 @@
 // chunk's codes in the upper half of its 128-byte row slots (a view of the
 // codes whose chunks are 64 bytes apart, started 64 bytes early), and the
 // page's 64 scales come with it; two groups of four converter warps (even and
-// odd pages) widen the codes in place to bf16 values equal to the codes, and
-// three more warps widen the peer tokens' value chunks the value warp loads the
-// same way.  Each group signals the leader's barrier once per CTA.  The scales
-// are applied in the softmax: to each token's score, and to its probability
-// before P goes to PV (a power of two: exact in bf16).
+// odd pages) widen the codes in place to bf16 values code * scale, exactly,
+// and three more warps widen the peer tokens' value chunks the value warp loads
+// the same way.  Each group signals the leader's barrier once per CTA.  The
+// softmax, the MMAs and the epilogue are those of the bf16 cache.
 //
 // The method is that of the single-CTA kernel ("FlashMLA: Revolutionizing
 // Efficient Decoding...", sections 4.2.1-4.2.3: TMA prefetch of 64-row latent
@@ -112,9 +111,6 @@ constexpr int kFp8RegsSoftmax = 176, kFp8RegsConv = 64;
 static_assert(128 * kFp8RegsSoftmax + 128 * kFp8LaunchRegs + 384 * kFp8RegsConv <=
                   640 * kFp8LaunchRegs,
               "FP8 setmaxnreg split within the launch's registers");
-// bf16 2^120: widened codes are code * 2^120 * 2^-120 = the code itself; each
-// token's scale is applied to its scores and probabilities instead
-constexpr uint32_t kBf16x2Pow120 = 0x7B807B80u;
 
 constexpr int kChunk = 64 * 128;          // 64 rows x 64 bf16 (one 128-byte swizzle column block)
 constexpr int kHalfChunk = 32 * 128;      // 32 rows x 64 bf16
@@ -270,25 +266,21 @@ __device__ __forceinline__ bool convert_wait(uint64_t* landed, uint32_t parity,
   return *abort_flag == 0;
 }
 
-// Widen one 128-byte row slot in place: its 64 E4M3 codes (bytes 64..127, as
-// the TMA box landed them) become the 64 codes as bf16 values over the whole
-// slot, in the 128-byte-swizzled layout (16-byte unit u of row r at (u ^ (r %
-// 8)) * 16).  For a code b = s eeee mmm the 16-bit pattern s 0000 eeee mmm 0000
-// is the bf16 value b * 2^-120 (E4M3 subnormals become bf16 subnormals); one
-// bf16x2 multiply by 2^120 makes it b, exactly.  A pattern is never NaN or
-// infinite, so rows past a sequence's end hold finite values (their scores are
-// masked and their probabilities are zero).  The four 16-byte loads start at
-// unit (r mod 4), so the lanes of a warp spread over the banks.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_codes(uint32_t word, uint32_t sel) {
-  const uint32_t t = __byte_perm(word, 0u, sel);  // (b_hi << 24) | (b_lo << 8)
-  const uint32_t pat = ((t & 0x7F007F00u) >> 4) | (t & 0x80008000u);
-  const uint32_t f = kBf16x2Pow120;
-  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pat);
-  v = __hmul2(v, *reinterpret_cast<const __nv_bfloat162*>(&f));
-  return *reinterpret_cast<const uint32_t*>(&v);
+// 2^60 * scale as bf16x2 (the scale is a power of two: its fp32 bits end in 16
+// zeros), or 0 for a row past the sequence's end (which must not reach an MMA:
+// its codes and scale may be anything).
+__device__ __forceinline__ uint32_t fp8_row_factor(bool row_ok, float scale) {
+  return row_ok ? (__float_as_uint(scale * 0x1p60f) >> 16) * 0x10001u : 0u;
 }
 
-__device__ __forceinline__ void widen_row_slot(uint8_t* slot, int r) {
+// Widen one 128-byte row slot in place: its 64 E4M3 codes (bytes 64..127, as
+// the TMA box landed them) become the 64 bf16 values code * scale over the
+// whole slot, in the 128-byte-swizzled layout (16-byte unit u of row r at
+// (u ^ (r % 8)) * 16); f_lo is fp8_row_factor of the row (see
+// e4m3x2_to_bf16x2: every step is exact).  The four 16-byte loads start at
+// unit (r mod 4), so the lanes of a warp spread over the banks.
+__device__ __forceinline__ void widen_row_slot(uint8_t* slot, int r, uint32_t f_lo) {
+  constexpr uint32_t f_hi = 0x5D805D80u;  // 2^60 in both halves
   uint4 v[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k)
@@ -297,14 +289,14 @@ __device__ __forceinline__ void widen_row_slot(uint8_t* slot, int r) {
   for (int k = 0; k < 4; ++k) {
     const int kk = (k + r) & 3;  // v[k] holds dims 16 kk .. 16 kk + 15 of the chunk
     uint4 lo, hi;
-    lo.x = e4m3x2_to_bf16x2_codes(v[k].x, 0x1404u);
-    lo.y = e4m3x2_to_bf16x2_codes(v[k].x, 0x3424u);
-    lo.z = e4m3x2_to_bf16x2_codes(v[k].y, 0x1404u);
-    lo.w = e4m3x2_to_bf16x2_codes(v[k].y, 0x3424u);
-    hi.x = e4m3x2_to_bf16x2_codes(v[k].z, 0x1404u);
-    hi.y = e4m3x2_to_bf16x2_codes(v[k].z, 0x3424u);
-    hi.z = e4m3x2_to_bf16x2_codes(v[k].w, 0x1404u);
-    hi.w = e4m3x2_to_bf16x2_codes(v[k].w, 0x3424u);
+    lo.x = e4m3x2_to_bf16x2(v[k].x, 0x1404u, f_hi, f_lo);
+    lo.y = e4m3x2_to_bf16x2(v[k].x, 0x3424u, f_hi, f_lo);
+    lo.z = e4m3x2_to_bf16x2(v[k].y, 0x1404u, f_hi, f_lo);
+    lo.w = e4m3x2_to_bf16x2(v[k].y, 0x3424u, f_hi, f_lo);
+    hi.x = e4m3x2_to_bf16x2(v[k].z, 0x1404u, f_hi, f_lo);
+    hi.y = e4m3x2_to_bf16x2(v[k].z, 0x3424u, f_hi, f_lo);
+    hi.z = e4m3x2_to_bf16x2(v[k].w, 0x1404u, f_hi, f_lo);
+    hi.w = e4m3x2_to_bf16x2(v[k].w, 0x3424u, f_hi, f_lo);
     *reinterpret_cast<uint4*>(slot + (((2 * kk) ^ (r & 7)) << 4)) = lo;
     *reinterpret_cast<uint4*>(slot + (((2 * kk + 1) ^ (r & 7)) << 4)) = hi;
   }
@@ -690,6 +682,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int pc = 0; pc < npieces; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       if (pz.npg == 0) continue;
+      const int L = p.seqlens[pz.seq];
       entries += 2;  // the query staging entries go straight to the consumers
       bool stop = false;
       for (int j = 0; j < pz.npg; ++j, ++entries) {
@@ -703,7 +696,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           break;
         }
         uint8_t* row_slot = sk + slot * kKBytes + r * 128;
-        for (int c = c0; c < kChunks; c += 4) widen_row_slot(row_slot + c * kHalfChunk, r);
+        const int tok = 32 * static_cast<int>(rank) + r;  // this CTA's token of the page
+        const uint32_t f_lo =
+            fp8_row_factor((pz.pg0 + j) * kPage + tok < L, sscale[slot * kPage + tok]);
+        for (int c = c0; c < kChunks; c += 4) widen_row_slot(row_slot + c * kHalfChunk, r, f_lo);
         fence_proxy_async_smem();  // the MMAs read the slot through the async proxy
         named_bar_sync(named, kKConvThreads);
         if (ct == 0) {
@@ -719,20 +715,27 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (kFp8 && warp >= kVConvWarp0) {
     // ------------------------------------------------------------ FP8: value converters
     // Widen the peer tokens' value chunks: 4 chunks x 32 rows, row slot i
-    // (row i % 32 of chunk i / 32) for i = t and t + 96.
+    // (row i % 32 of chunk i / 32) for i = t and t + 96.  The tokens' scales
+    // came with this CTA's K part: its landed barrier (still in this page's
+    // phase: the slot is not reloaded before PV of the page, which waits for
+    // these converters) makes them visible here.
     const int ct = threadIdx.x - kVConvWarp0 * 32;
     const int dst_chunk = rank == 0 ? kXChunks : 0;
+    const int src_row = rank == 0 ? 32 : 0;
     int entries = 0;
-    uint32_t landed_parity = 0;
+    uint32_t landed_parity = 0, k_parity = 0;
     for (int pc = 0; pc < npieces; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       if (pz.npg == 0) continue;
+      const int L = p.seqlens[pz.seq];
       entries += 2;
       bool stop = false;
       for (int j = 0; j < pz.npg; ++j, ++entries) {
         const int slot = entries % kKSlots;
-        const uint32_t parity = (landed_parity >> slot) & 1;
+        const uint32_t parity = (landed_parity >> slot) & 1, kpar = (k_parity >> slot) & 1;
         landed_parity ^= 1u << slot;
+        k_parity ^= 1u << slot;
+        mbar_wait(&bar[kKLanded0 + slot], kpar, abort_flag, wait_ns);
         if (!convert_wait(&bar[kVLanded0 + slot], parity, abort_flag, wait_ns, kVConvBarrier,
                           kVConvThreads)) {
           stop = true;
@@ -740,7 +743,10 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         for (int i = ct; i < kXChunks * 32; i += kVConvThreads) {
           const int r = i & 31;
-          widen_row_slot(sk + slot * kKBytes + (dst_chunk + (i >> 5)) * kHalfChunk + r * 128, r);
+          const uint32_t f_lo = fp8_row_factor((pz.pg0 + j) * kPage + src_row + r < L,
+                                               sscale[slot * kPage + src_row + r]);
+          widen_row_slot(sk + slot * kKBytes + (dst_chunk + (i >> 5)) * kHalfChunk + r * 128, r,
+                         f_lo);
         }
         fence_proxy_async_smem();
         named_bar_sync(kVConvBarrier, kVConvThreads);
@@ -908,7 +914,6 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     int entries = 0, pages = 0, pieces_done = 0, qcopies = 0;
     bool ok = true;
     bool q_copied_ahead = false;
-    uint32_t landed_parity = 0;  // FP8: per slot, pages whose codes and scales landed (mod 2)
     for (int pc = 0; pc < npieces && ok; ++pc) {
       const Piece pz = piece_of(md, pc, p.seqlens, p.bt_stride);
       const int Lseq = p.seqlens[pz.seq];
@@ -939,25 +944,11 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           tc_fence_before();
           warp_arrive_leader(&bar[kSFree0 + pb], rank, lane);
           const int nv = lim - (pz.pg0 + j) * kPage - 32 * th;
-          // FP8 cache: the MMAs saw the codes; token c's scale multiplies its
-          // score here and its probability below.  The page's scales landed with
-          // this CTA's K part (the barrier's phase is complete: the slot is not
-          // reloaded before PV of this page, which needs this softmax).
-          const float* tsc = sscale;  // FP8: this thread's 32 tokens' scales
-          if constexpr (kFp8) {
-            const int slot = (entries + j) % kKSlots;
-            const uint32_t parity = (landed_parity >> slot) & 1;
-            landed_parity ^= 1u << slot;
-            ok = warp_wait_cluster(&bar[kKLanded0 + slot], parity, abort_flag, wait_ns);
-            if (!ok) break;
-            tsc = sscale + slot * kPage + 32 * th;
-          }
           float x[32];
           float mx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float sc = kFp8 ? p.scale_log2 * tsc[c] : p.scale_log2;
-            x[c] = c < nv ? __uint_as_float(s[c]) * sc : -INFINITY;
+            x[c] = c < nv ? __uint_as_float(s[c]) * p.scale_log2 : -INFINITY;
             mx = fmaxf(mx, x[c]);
           }
           // the other half of the row is in lane L ^ 64
@@ -979,14 +970,7 @@ mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             const float p0 = x[c] == -INFINITY ? 0.f : ex2_approx(x[c] - m);
             const float p1 = x[c + 1] == -INFINITY ? 0.f : ex2_approx(x[c + 1] - m);
             sum += p0 + p1;
-            if constexpr (kFp8) {
-              // the value rows are the codes: P carries the scale (a power of
-              // two, so the bf16 rounding of P is unchanged); a masked token
-              // keeps P = 0 whatever its scale holds
-              pw[c >> 1] = pack_bf16x2(p0 == 0.f ? 0.f : p0 * tsc[c], p1 == 0.f ? 0.f : p1 * tsc[c + 1]);
-            } else {
-              pw[c >> 1] = pack_bf16x2(p0, p1);
-            }
+            pw[c >> 1] = pack_bf16x2(p0, p1);
           }
           l = l * alpha + sum;
           // O is rescaled only once PV of the previous page is done; the first

@@ -120,9 +120,8 @@ def test_fp8_decode_forced_splits(cuda_device, num_workers, h_q):
 @pytest.mark.parametrize("h_q", [16, 128])
 def test_fp8_decode_ignores_stale_tail_rows(cuda_device, h_q):
     # rows past each sequence's end hold NaN codes and infinite scales: the
-    # kernel must never let them reach an output (16 heads: single CTAs, which
-    # zero such rows; 128 heads: CTA pairs, which mask their scores and give
-    # them zero probability whatever their scale holds)
+    # kernels must never let them reach an output (16 heads: single CTAs; 128
+    # heads: CTA pairs)
     w = synth.custom_workload(3, 1, h_q, [37, 64, 100])
     inp = synth.make_inputs(w, seed=32)
     codes, scales = encode_cache(inp.kcache)
