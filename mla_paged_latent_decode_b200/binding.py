@@ -248,13 +248,17 @@ def mla_decode_kvcache(q: torch.Tensor, kcache: torch.Tensor, block_table: torch
     return out, lse
 
 
-def _check_state(block_table, cache_seqlens, free_pages, free_count, dev):
+def _check_state(block_table, cache_seqlens, free_pages, free_count, dev, device_status=None):
     for t in (block_table, cache_seqlens, free_pages, free_count):
         _require(t.is_cuda and t.device == dev and t.is_contiguous() and t.dtype == torch.int32,
                  "page-state tensors must be contiguous int32 on one CUDA device")
     _require(block_table.dim() == 2 and block_table.shape[0] == cache_seqlens.numel(),
              "block_table must be [batch, max_pages]")
     _require(free_count.numel() == 1, "free_count must hold one int32")
+    if device_status is not None:
+        _require(device_status.dtype == torch.int32 and device_status.numel() >= 1 and
+                 device_status.is_contiguous() and device_status.device == dev,
+                 "device_status must hold one int32 on the cache's device")
 
 
 def append_latent(rows: torch.Tensor, kcache: torch.Tensor, block_table: torch.Tensor,
@@ -271,7 +275,7 @@ def append_latent(rows: torch.Tensor, kcache: torch.Tensor, block_table: torch.T
              "rows and kcache must be contiguous on one device")
     _require(kcache.dim() == 3 and kcache.shape[1] == PAGE and kcache.shape[2] == d == D_QK,
              "kcache must be [num_blocks, 64, 576] and rows [batch, s_new, 576]")
-    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev, device_status)
     _require(cache_seqlens.numel() == b, "cache_seqlens must have one entry per sequence")
     with torch.cuda.device(dev):
         _check(lib.mla_append_latent(_ptr(rows), s_new, _ptr(kcache), kcache.shape[0],
@@ -287,7 +291,7 @@ def release_pages(release_mask: torch.Tensor, block_table: torch.Tensor,
     """Push the pages of every sequence with release_mask[i] != 0 back onto the free stack and
     set its length to 0 (in place, on the current stream)."""
     dev = cache_seqlens.device
-    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev, device_status)
     _require(release_mask.dtype == torch.int32 and release_mask.device == dev,
              "release_mask must be int32 on the cache's device")
     _require(release_mask.is_contiguous() and release_mask.numel() == cache_seqlens.numel(),
@@ -314,10 +318,10 @@ def append_latent_fp8(rows: torch.Tensor, kcache8: torch.Tensor, kscale: torch.T
              "kcache8 must be contiguous uint8 on the rows' device")
     _require(kcache8.dim() == 3 and kcache8.shape[1] == PAGE and kcache8.shape[2] == D_QK,
              "kcache8 must be [num_blocks, 64, 576]")
-    _require(kscale.dtype == torch.float32 and kscale.is_contiguous(),
-             "kscale must be contiguous fp32")
+    _require(kscale.dtype == torch.float32 and kscale.is_contiguous() and kscale.device == dev,
+             "kscale must be contiguous fp32 on the rows' device")
     _require(tuple(kscale.shape) == tuple(kcache8.shape[:2]), "kscale must be [num_blocks, 64]")
-    _check_state(block_table, cache_seqlens, free_pages, free_count, dev)
+    _check_state(block_table, cache_seqlens, free_pages, free_count, dev, device_status)
     _require(cache_seqlens.numel() == b, "cache_seqlens must have one entry per sequence")
     with torch.cuda.device(dev):
         _check(lib.mla_append_latent_fp8(_ptr(rows), s_new, _ptr(kcache8), _ptr(kscale),

@@ -341,3 +341,39 @@ def test_merge_host_validation():
                dict(out=(1 << 13) + 8), dict(lse=(1 << 13) + 2), dict(s_q=512, h_q=256),
                dict(R=4096, b=1 << 16, h_q=128)):
         assert call(**kw) == binding.MLA_ERR_INVALID_ARG, kw
+
+
+@pytest.mark.parametrize("bad,match", [
+    ("rows_fp32", "rows must be contiguous bf16"),
+    ("codes_bf16", "kcache8 must be contiguous uint8"),
+    ("codes_page", r"kcache8 must be \[num_blocks, 64, 576\]"),
+    ("scale_fp16", "kscale must be contiguous fp32"),
+    ("scale_device", "kscale must be contiguous fp32 on the rows' device"),
+    ("scale_short", r"kscale must be \[num_blocks, 64\]"),
+])
+def test_fp8_append_checks_codes_and_scales(bad, match):
+    # the FP8 append writes codes and scales through raw pointers: every extent,
+    # type and device is checked before the call
+    import torch
+    b, nb = 2, 4
+    rows = torch.zeros((b, 3, 576), dtype=torch.bfloat16)
+    codes = torch.zeros((nb, 64, 576), dtype=torch.uint8)
+    scales = torch.ones((nb, 64), dtype=torch.float32)
+    if bad == "rows_fp32":
+        rows = rows.float()
+    elif bad == "codes_bf16":
+        codes = codes.to(torch.bfloat16)
+    elif bad == "codes_page":
+        codes = torch.zeros((nb, 32, 576), dtype=torch.uint8)
+    elif bad == "scale_fp16":
+        scales = scales.half()
+    elif bad == "scale_device":
+        scales = torch.ones((nb, 64), dtype=torch.float32, device="meta")
+    elif bad == "scale_short":
+        scales = scales[:, :32].contiguous()
+    with pytest.raises(ValueError, match=match):
+        binding.append_latent_fp8(rows, codes, scales,
+                                  torch.zeros((b, 3), dtype=torch.int32),
+                                  torch.zeros(b, dtype=torch.int32),
+                                  torch.arange(nb, dtype=torch.int32),
+                                  torch.tensor([nb], dtype=torch.int32))
