@@ -172,3 +172,26 @@ def test_grid_rounding_equals_table_rounding():
     rand = rand[rand <= 448] * np.where(g.random(rand.size) < 0.5, -1, 1)
     for y in (vals, mids, -mids, rand, np.array([0.0, -0.0, 2.0 ** -12, -2.0 ** -12])):
         np.testing.assert_array_equal(f8.e4m3_round_grid(y), f8.e4m3_round(y))
+
+
+def test_format_agrees_with_torch_float8_e4m3fn():
+    # an independent implementation of the same format (OCP E4M3, "fn": no
+    # infinities, NaN at S.1111.111): every code's value, and nearest-even
+    # rounding of float32 values inside the range, including exact midpoints
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib_vals = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = f8.decode_codes(codes.numpy())
+    finite = ~np.isnan(lib_vals)
+    assert finite.sum() == 254
+    np.testing.assert_array_equal(np.isnan(ours), ~finite)
+    np.testing.assert_array_equal(ours[finite], lib_vals[finite])
+    np.testing.assert_array_equal(np.signbit(ours[finite]), np.signbit(lib_vals[finite]))
+
+    g = np.random.default_rng(7)
+    mags = np.ldexp(g.random(20000) + 0.5, g.integers(-14, 9, size=20000)).astype(np.float32)
+    vals = np.sort(f8.decode_codes(np.arange(0x00, 0x7F)))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)      # exact in float32
+    ys = np.concatenate([mags, -mags, mids, -mids]).astype(np.float32)
+    ys = ys[np.abs(ys) <= 448]
+    lib_codes = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(f8.e4m3_round(ys.astype(np.float64)), lib_codes)
