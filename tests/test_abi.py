@@ -377,3 +377,27 @@ def test_fp8_append_checks_codes_and_scales(bad, match):
                                   torch.zeros(b, dtype=torch.int32),
                                   torch.arange(nb, dtype=torch.int32),
                                   torch.tensor([nb], dtype=torch.int32))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # no fallback: without the built library the binding refuses to import
+    import sys
+    env = dict(os.environ, MLA_DECODE_LIB=str(tmp_path / "absent.so"))
+    r = subprocess.run([sys.executable, "-c", "import mla_paged_latent_decode_b200.binding"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "not built" in r.stderr
+
+
+def test_product_code_never_reaches_the_oracle():
+    # the package and the C ABI neither import nor link anything under oracle/
+    pkg = os.path.join(ROOT, "mla_paged_latent_decode_b200")
+    pat = re.compile(r"^\s*(import\s+oracle|from\s+oracle\b|#include\s+[<\"].*oracle)", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, name)) as f:
+                    assert not pat.search(f.read()), name
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        with open(os.path.join(ROOT, "include", name)) as f:
+            assert not pat.search(f.read()), name
